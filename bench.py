@@ -1,0 +1,371 @@
+#!/usr/bin/env python
+"""Benchmark of the Longformer attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload base_bf16]
+
+One step = one forward pass of the whole attention (mask pass, global-token
+gathers, the fused band + global-row tensor-core kernel and the split
+combine) over one batch of the workload, inputs resident in HBM.  The timed
+region is K steps between a barrier + synchronize on both sides, timed with
+CUDA events on the launching stream; the max over ranks is reported.  The
+inputs rotate over several buffer sets whose total exceeds the L2 cache, so
+no step reads another step's inputs out of L2.
+
+Metric: attended scores per second (and TFLOP/s at 4 * head_dim FLOP per
+attended pair), whole job.  Multi-GPU (torchrun): every rank runs its own
+copy of the workload (independent batches, no collective on the data path):
+weak scaling.
+
+--impl reference times the CPU oracle (oracle/, float64, OpenMP) on a
+bounded sample of the same workload -- the only reference implementation
+this project has (the pages publish no code to install).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_sliding_window_b200 import synth  # noqa: E402
+
+METRIC = "attended scores/s and TFLOP/s at n=4096 w=512 bf16; % of B200 roofline"
+UNIT = "scores/s"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        j = json.load(open(path))
+        return dict(hbm=float(j["hbm_gbs"]), bf16=float(j["bf16_tflops"]),
+                    bf16_sus=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def algorithmic_bytes(wl, mask) -> int:
+    """Bytes one forward must move at least: Q_s, K_s, V_s read and O
+    written for every row, Q_g read at the global rows, K_g and V_g read in
+    full, the mask read and the fp32 log-normaliser written."""
+    eb = 4 if wl.dtype == "f32" else 2
+    row = wl.head_dim * eb
+    nrows = wl.B * wl.H * wl.n
+    ng = int((mask == 2).sum())
+    return (4 * nrows * row + wl.H * ng * row + 2 * nrows * row + mask.size * 4 + nrows * 4)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_uuid=None):
+        self.proc = None
+        self.out = None
+        self.uuid = dev_uuid
+
+    def start(self):
+        try:
+            cmd = ["nvidia-smi", "--query-gpu=" + self.Q, "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.out = open(os.path.join("/tmp", "lf_clocks_%d.csv" % os.getpid()), "w+")
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.seek(0)
+        rows = [l.strip().split(",") for l in self.out if l.strip()]
+        self.out.close()
+        try:
+            os.remove(self.out.name)
+        except OSError:
+            pass
+        sm, mx, reasons, pw = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                pw.append(float(r[3]))
+                for k, nm in enumerate(names):
+                    if r[5 + k].strip().lower() == "active":
+                        reasons.add(nm)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "power_w_max": float(max(pw)) if pw else None, "reasons": sorted(reasons),
+                "samples": len(sm), "window": "warm-up and timed region"}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args, wl):
+    """The CPU oracle on a bounded sample (whole heads) of the workload."""
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    inp = synth.make_inputs(wl)
+    f = {k: synth.as_float64(v, wl.dtype) for k, v in inp.items() if k not in ("mask", "dilation")}
+    scale = 1.0 / math.sqrt(wl.head_dim)
+    head = (0, 0)
+    pairs = oracle.count_pairs(wl.n, wl.r, wl.dilation[0], wl.causal, inp["mask"][0])
+
+    def step():
+        b, h = head
+        oracle.fwd_head(wl.r, wl.dilation[h], wl.causal, scale, inp["mask"][b], f["qs"][b, h],
+                        f["ks"][b, h], f["vs"][b, h], f["qg"][b, h], f["kg"][b, h], f["vg"][b, h])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    v = pairs / dt
+    sample = "one (b,h) head of %s per step (%d of %d heads)" % (wl.name, 1, wl.B * wl.H)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "n": wl.n,
+                                            "window": 2 * wl.r, "head_dim": wl.head_dim},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(wl, budget_s=10.0):
+    """The oracle as it stands, timed on the host cores over whole heads of
+    the workload until ~budget_s seconds of work (rank 0, N = 1 only)."""
+    import oracle
+    oracle.build()
+    inp = synth.make_inputs(wl)
+    f = {k: synth.as_float64(v, wl.dtype) for k, v in inp.items() if k not in ("mask", "dilation")}
+    scale = 1.0 / math.sqrt(wl.head_dim)
+    done, pairs, t_total = 0, 0, 0.0
+    for b in range(wl.B):
+        for h in range(wl.H):
+            t0 = time.perf_counter()
+            oracle.fwd_head(wl.r, wl.dilation[h], wl.causal, scale, inp["mask"][b], f["qs"][b, h],
+                            f["ks"][b, h], f["vs"][b, h], f["qg"][b, h], f["kg"][b, h], f["vg"][b, h])
+            t_total += time.perf_counter() - t0
+            pairs += oracle.count_pairs(wl.n, wl.r, wl.dilation[h], wl.causal, inp["mask"][b])
+            done += 1
+            if t_total >= budget_s:
+                break
+        if t_total >= budget_s:
+            break
+    return {"value": pairs / t_total, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": "%d of %d (b,h) heads of %s, float64, %.1f s" % (done, wl.B * wl.H, wl.name, t_total)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="base_bf16", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--min-warm-seconds", type=float, default=1.0)
+    args = ap.parse_args()
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    import torch
+    from sparse_sliding_window_b200 import lf_attn as L
+
+    world, rank, local = _dist()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    kern = {"auto": L.LF_KERNEL_AUTO, "simt": L.LF_KERNEL_SIMT, "tc": L.LF_KERNEL_TC}[args.kernel]
+
+    inp = synth.make_inputs(wl, with_do=False)
+    mask_np = inp["mask"]
+    ng = int((mask_np == 2).sum(axis=1).max())
+    att = L.LongformerAttention(wl.B, wl.H, wl.n, wl.r, wl.dilation, wl.causal, dtype=wl.dtype,
+                                max_global=ng, kernel=kern, device=dev)
+    tdt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[wl.dtype]
+
+    def host_tensor(a):
+        if wl.dtype == "bf16":
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(a)
+
+    names = ["qs", "ks", "vs", "qg", "kg", "vg"]
+    host = {k: host_tensor(inp[k]).pin_memory() for k in names}
+    host["mask"] = torch.from_numpy(mask_np).pin_memory()
+    set_bytes = sum(host[k].numel() * host[k].element_size() for k in names)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    nsets = max(2, int(math.ceil(1.5 * l2 / max(set_bytes, 1))) + 1)
+    sets = []
+    for s in range(nsets):
+        d = {k: host[k].to(dev, non_blocking=False) for k in names + ["mask"]}
+        d["o"] = torch.empty_like(d["qs"])
+        d["lse"] = torch.empty(d["qs"].shape[:3], dtype=torch.float32, device=dev)
+        sets.append(d)
+    torch.cuda.synchronize(dev)
+
+    # attended pairs of one step, from the library's pair counter (exact
+    # against the oracle in tests/)
+    pairs = int(att.count_pairs(sets[0]["mask"]).sum().item())
+    att.status()
+
+    def step(i):
+        d = sets[i % nsets]
+        att.fwd(d["qs"], d["ks"], d["vs"], d["qg"], d["kg"], d["vg"], d["mask"], d["o"], d["lse"])
+
+    # warm-up (count-based, stretched to >= min_warm_seconds for the clock samples)
+    sampler = ClockSampler(getattr(torch.cuda.get_device_properties(dev), "uuid", None) and
+                           "GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    sampler.start()
+    i = 0
+    t_start = time.time()
+    while i < args.warmup or time.time() - t_start < args.min_warm_seconds:
+        step(i)
+        i += 1
+        if i % 64 == 0:
+            torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(dev)
+    att.status()
+
+    # kernel timing events (main attention kernel of every timed step)
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = L.lf_attn_launch_count()
+    e0.record(stream)
+    for k in range(args.steps):
+        L.lf_attn_set_timing_events(*kev[k])
+        step(i + k)
+    e1.record(stream)
+    L.lf_attn_set_timing_events(None, None)
+    torch.cuda.synchronize(dev)
+    launches = L.lf_attn_launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    t_ms = e0.elapsed_time(e1)
+    k_ms = float(np.mean([a.elapsed_time(b) for a, b in kev]))
+    att.status()
+    if world > 1:
+        t = torch.tensor([t_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_ms = float(t.item())
+    ms_step = t_ms / args.steps
+    value = pairs * world / (ms_step * 1e-3)
+    flops = 4.0 * wl.head_dim * pairs
+    tflops = flops * world / (ms_step * 1e-3) / 1e12
+
+    # end-to-end through the public API: H2D of the step's inputs from pinned
+    # host memory, the forward, D2H of the output
+    o_host = torch.empty(sets[0]["o"].shape, dtype=tdt).pin_memory()
+    d = sets[0]
+    for _ in range(3):
+        for k in names + ["mask"]:
+            d[k].copy_(host[k], non_blocking=True)
+        att.fwd(d["qs"], d["ks"], d["vs"], d["qg"], d["kg"], d["vg"], d["mask"], d["o"], d["lse"])
+        o_host.copy_(d["o"], non_blocking=True)
+    torch.cuda.synchronize(dev)
+    ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 50))
+    ee0.record(stream)
+    for _ in range(e2e_steps):
+        for k in names + ["mask"]:
+            d[k].copy_(host[k], non_blocking=True)
+        att.fwd(d["qs"], d["ks"], d["vs"], d["qg"], d["kg"], d["vg"], d["mask"], d["o"], d["lse"])
+        o_host.copy_(d["o"], non_blocking=True)
+    ee1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = ee0.elapsed_time(ee1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = set_bytes + host["mask"].numel() * 4
+    d2h = o_host.numel() * o_host.element_size()
+
+    pk = _peaks()
+    abytes = algorithmic_bytes(wl, mask_np)
+    t_flop = flops / (pk["bf16"] * 1e12)
+    t_byte = abytes / (pk["hbm"] * 1e9)
+    k_s = k_ms * 1e-3
+    if t_byte >= t_flop:
+        roof = {"bound": "hbm", "achieved": abytes / k_s / 1e9, "peak": pk["hbm"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / k_s / 1e12, "peak": pk["bf16"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["peak_source"] = pk["src"]
+    roof["kernel_ms"] = k_ms
+    roof["algorithmic_bytes"] = abytes
+    roof["algorithmic_flops"] = flops
+    roof["tensor_view"] = {"achieved_tflops": flops / k_s / 1e12, "peak": pk["bf16"],
+                           "frac": flops / k_s / 1e12 / pk["bf16"]}
+    roof["step_frac"] = max(t_flop, t_byte) / (ms_step * 1e-3)
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "n": wl.n, "window": 2 * wl.r,
+                       "head_dim": wl.head_dim, "dilation": sorted(set(wl.dilation)),
+                       "causal": wl.causal, "global_tokens_per_seq": ng, "kernel": args.kernel,
+                       "l2": "inputs rotate over %d buffer sets (%.0f MB > L2 %.0f MB)" % (
+                           nsets, nsets * set_bytes / 1e6, l2 / 1e6),
+                       "parallelism": "replicas x%d" % world if world > 1 else "1 GPU"},
+            "tflops": tflops, "attended_pairs_per_step": pairs * world,
+            "roofline": roof, "clocks": clocks, "gpu_launches": int(launches),
+            "e2e": {"value": pairs * world / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                    "ms_per_step": e2e_ms}}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,256 @@
+// lf_api.cu -- the C ABI (include/lf_attn.h): argument validation, the
+// workspace carve-up, and the launch sequence of each call on the caller's
+// stream.  No call allocates device memory; every device buffer, including
+// the workspace, belongs to the caller.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <atomic>
+
+#include "lf_attn.h"
+#include "lf_common.cuh"
+#include "lf_tc.cuh"
+
+static thread_local char g_err[512];
+static std::atomic<uint64_t> g_launches{0};
+
+void lf_launches_add(int k) { g_launches.fetch_add((uint64_t)k, std::memory_order_relaxed); }
+uint64_t lf_launches_get() { return g_launches.load(std::memory_order_relaxed); }
+static thread_local cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
+
+static int lf_fail(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+static int lf_cuda(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return LF_OK;
+  return lf_fail(LF_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+extern "C" int lf_attn_version(void) { return 1; }
+
+extern "C" uint64_t lf_attn_launch_count(void) { return lf_launches_get(); }
+
+extern "C" const char *lf_attn_last_error(void) { return g_err; }
+
+extern "C" int lf_attn_set_timing_events(void *ev_start, void *ev_stop) {
+  g_ev_start = (cudaEvent_t)ev_start;
+  g_ev_stop = (cudaEvent_t)ev_stop;
+  return LF_OK;
+}
+
+static size_t lf_align(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static size_t lf_dtype_bytes(int dt) { return dt == LF_F32 ? 4 : 2; }
+
+// Validate params; fill the device block and the workspace layout.
+static int lf_prepare(const lf_attn_params *p, int for_bwd, LfDev &dev, LfWs &ws) {
+  g_err[0] = 0;
+  if (!p) return lf_fail(LF_ERR_INVALID, "params is NULL");
+  if (p->B < 1 || p->H < 1 || p->n < 1)
+    return lf_fail(LF_ERR_INVALID, "B, H, n must be >= 1 (got %d, %d, %d)", p->B, p->H, p->n);
+  if (p->H > LF_MAX_H) return lf_fail(LF_ERR_UNSUPPORTED, "H = %d > %d", p->H, LF_MAX_H);
+  if (p->head_dim != LF_HD) return lf_fail(LF_ERR_UNSUPPORTED, "head_dim must be 64 (got %d)", p->head_dim);
+  if (p->window < 0) return lf_fail(LF_ERR_INVALID, "window must be >= 0 (got %d)", p->window);
+  if (p->causal != 0 && p->causal != 1) return lf_fail(LF_ERR_INVALID, "causal must be 0 or 1");
+  if (p->dtype < LF_F32 || p->dtype > LF_F16) return lf_fail(LF_ERR_INVALID, "bad dtype %d", p->dtype);
+  if (p->kernel < LF_KERNEL_AUTO || p->kernel > LF_KERNEL_TC)
+    return lf_fail(LF_ERR_INVALID, "bad kernel selector %d", p->kernel);
+  if (p->kernel == LF_KERNEL_TC && p->dtype == LF_F32)
+    return lf_fail(LF_ERR_UNSUPPORTED, "the tensor-core path takes bf16 or f16, not f32");
+  if (!(p->scale >= 0.f) || isinf(p->scale)) return lf_fail(LF_ERR_INVALID, "scale must be finite and >= 0");
+  if ((long long)p->B * p->H * p->n > (1ll << 31) - 64)
+    return lf_fail(LF_ERR_UNSUPPORTED, "B*H*n too large");
+  memset(&dev, 0, sizeof(dev));
+  const int n = p->n;
+  int dmax = 1;
+  for (int h = 0; h < p->H; h++) {
+    int d = p->dilation ? p->dilation[h] : 1;
+    if (d < 1) return lf_fail(LF_ERR_INVALID, "dilation[%d] = %d < 1", h, d);
+    d = std::min(d, n);  // d >= n keeps only k = 0: same pattern as d = n
+    dev.dil[h] = d;
+    dmax = std::max(dmax, d);
+  }
+  // a window past the sequence end is the same as one that just reaches it
+  const int r = std::min(p->window, n);
+  if ((long long)r * dmax + n >= (1ll << 30))
+    return lf_fail(LF_ERR_UNSUPPORTED, "window * dilation too large");
+  const int G = p->max_global < 0 ? n : std::min(p->max_global, n);
+  dev.B = p->B;
+  dev.H = p->H;
+  dev.n = n;
+  dev.r = r;
+  dev.causal = p->causal;
+  dev.G = G;
+  dev.Gk = (G + 15) / 16 * 16;
+  dev.scale = p->scale > 0.f ? p->scale : 1.f / sqrtf((float)p->head_dim);
+  dev.scale_log2 = dev.scale * LF_LOG2E;
+  dev.chunk_tiles = LF_TC_CHUNK_TILES;
+  dev.nch = (n + LF_BK * LF_TC_CHUNK_TILES - 1) / (LF_BK * LF_TC_CHUNK_TILES);
+
+  const size_t B = p->B, H = p->H, eb = lf_dtype_bytes(p->dtype);
+  const size_t Ga = std::max(G, 1), Gka = std::max(dev.Gk, 16);
+  size_t off = 0;
+  ws.status = off;
+  off = lf_align(off + LF_ST_WORDS * 4);
+  ws.binfo = off;
+  off = lf_align(off + B * LF_BI_WORDS * 4);
+  ws.gidx = off;
+  off = lf_align(off + B * Ga * 4);
+  const bool tc = p->dtype != LF_F32 && p->kernel != LF_KERNEL_SIMT;
+  ws.qg_c = ws.ks_c = ws.vs_c = ws.part_acc = ws.part_ml = off;
+  if (tc && !for_bwd) {
+    ws.qg_c = off;
+    off = lf_align(off + B * H * Ga * LF_HD * eb);
+    ws.ks_c = off;
+    off = lf_align(off + B * H * Gka * LF_HD * eb);
+    ws.vs_c = off;
+    off = lf_align(off + B * H * Gka * LF_HD * eb);
+    ws.part_acc = off;
+    off = lf_align(off + B * H * Ga * dev.nch * LF_HD * 4);
+    ws.part_ml = off;
+    off = lf_align(off + B * H * Ga * dev.nch * 8);
+  }
+  ws.delta = off;
+  if (for_bwd) off = lf_align(off + B * H * (size_t)n * 4);
+  ws.total = off;
+  ws.G = (int)Ga;
+  ws.Gk = (int)Gka;
+  ws.nch = dev.nch;
+  return LF_OK;
+}
+
+extern "C" size_t lf_attn_workspace_size(const lf_attn_params *p, int for_bwd) {
+  LfDev dev;
+  LfWs ws;
+  if (lf_prepare(p, for_bwd ? 1 : 0, dev, ws) != LF_OK) return 0;
+  return ws.total;
+}
+
+static int lf_check_ptr(const void *ptr, const char *name, bool may_be_null = false) {
+  if (!ptr) return may_be_null ? LF_OK : lf_fail(LF_ERR_INVALID, "%s is NULL", name);
+  if (((uintptr_t)ptr) & 15) return lf_fail(LF_ERR_INVALID, "%s is not 16-byte aligned", name);
+  return LF_OK;
+}
+
+static int lf_bind_ws(const lf_attn_params *p, int for_bwd, void *workspace, size_t ws_bytes,
+                      const int32_t *mask, void *stream, LfLaunch &L) {
+  int st = lf_prepare(p, for_bwd, L.dev, L.ws);
+  if (st) return st;
+  if (!workspace) return lf_fail(LF_ERR_INVALID, "workspace is NULL");
+  if (((uintptr_t)workspace) & 255) return lf_fail(LF_ERR_INVALID, "workspace is not 256-byte aligned");
+  if (ws_bytes < L.ws.total)
+    return lf_fail(LF_ERR_INVALID, "workspace too small: %zu < %zu bytes", ws_bytes, L.ws.total);
+  if ((st = lf_check_ptr(mask, "mask"))) return st;
+  L.ws_base = (char *)workspace;
+  L.stream = (cudaStream_t)stream;
+  L.dtype = p->dtype;
+  L.dev.mask = mask;
+  L.dev.status = (int32_t *)(L.ws_base + L.ws.status);
+  L.dev.binfo = (int32_t *)(L.ws_base + L.ws.binfo);
+  L.dev.gidx = (int32_t *)(L.ws_base + L.ws.gidx);
+  // each call starts with a clear status word; lf_attn_status reads it back
+  return lf_cuda(cudaMemsetAsync(L.dev.status, 0, LF_ST_WORDS * 4, L.stream), "status reset");
+}
+
+extern "C" int lf_attn_fwd(const lf_attn_params *p, const void *q_s, const void *k_s,
+                           const void *v_s, const void *q_g, const void *k_g, const void *v_g,
+                           const int32_t *mask, void *o, float *lse, void *workspace,
+                           size_t ws_bytes, void *stream) {
+  int st;
+  if ((st = lf_check_ptr(q_s, "q_s")) || (st = lf_check_ptr(k_s, "k_s")) ||
+      (st = lf_check_ptr(v_s, "v_s")) || (st = lf_check_ptr(q_g, "q_g")) ||
+      (st = lf_check_ptr(k_g, "k_g")) || (st = lf_check_ptr(v_g, "v_g")) ||
+      (st = lf_check_ptr(o, "o")) || (st = lf_check_ptr(lse, "lse", true)))
+    return st;
+  LfLaunch L;
+  if ((st = lf_bind_ws(p, 0, workspace, ws_bytes, mask, stream, L))) return st;
+  if ((st = lf_cuda(lf_launch_mask_pass(L), "mask pass"))) return st;
+  const bool tc = p->dtype != LF_F32 && p->kernel != LF_KERNEL_SIMT;
+  if (tc) {
+    LfTcArgs a{q_s, k_s, v_s, q_g, k_g, v_g, o, lse, g_ev_start, g_ev_stop};
+    st = lf_tc_fwd(L, a, g_err, sizeof(g_err));
+    if (st) return st;
+  } else {
+    if (g_ev_start && g_ev_stop) cudaEventRecord(g_ev_start, L.stream);
+    if ((st = lf_cuda(lf_launch_simt_fwd(L, q_s, k_s, v_s, q_g, k_g, v_g, o, lse), "forward")))
+      return st;
+    if (g_ev_start && g_ev_stop) cudaEventRecord(g_ev_stop, L.stream);
+  }
+  return LF_OK;
+}
+
+extern "C" int lf_attn_bwd(const lf_attn_params *p, const void *q_s, const void *k_s,
+                           const void *v_s, const void *q_g, const void *k_g, const void *v_g,
+                           const int32_t *mask, const void *o, const float *lse, const void *d_o,
+                           void *dq_s, void *dk_s, void *dv_s, void *dq_g, void *dk_g, void *dv_g,
+                           void *workspace, size_t ws_bytes, void *stream) {
+  int st;
+  if ((st = lf_check_ptr(q_s, "q_s")) || (st = lf_check_ptr(k_s, "k_s")) ||
+      (st = lf_check_ptr(v_s, "v_s")) || (st = lf_check_ptr(q_g, "q_g")) ||
+      (st = lf_check_ptr(k_g, "k_g")) || (st = lf_check_ptr(v_g, "v_g")) ||
+      (st = lf_check_ptr(o, "o")) || (st = lf_check_ptr(lse, "lse")) ||
+      (st = lf_check_ptr(d_o, "d_o")) || (st = lf_check_ptr(dq_s, "dq_s")) ||
+      (st = lf_check_ptr(dk_s, "dk_s")) || (st = lf_check_ptr(dv_s, "dv_s")) ||
+      (st = lf_check_ptr(dq_g, "dq_g")) || (st = lf_check_ptr(dk_g, "dk_g")) ||
+      (st = lf_check_ptr(dv_g, "dv_g")))
+    return st;
+  LfLaunch L;
+  if ((st = lf_bind_ws(p, 1, workspace, ws_bytes, mask, stream, L))) return st;
+  if ((st = lf_cuda(lf_launch_mask_pass(L), "mask pass"))) return st;
+  return lf_cuda(lf_launch_simt_bwd(L, q_s, k_s, v_s, q_g, k_g, v_g, o, lse, d_o, dq_s, dk_s, dv_s,
+                                    dq_g, dk_g, dv_g),
+                 "backward");
+}
+
+extern "C" int lf_attn_count_pairs(const lf_attn_params *p, const int32_t *mask, int64_t *counts,
+                                   void *workspace, size_t ws_bytes, void *stream) {
+  int st;
+  if ((st = lf_check_ptr(counts, "counts"))) return st;
+  LfLaunch L;
+  if ((st = lf_bind_ws(p, 0, workspace, ws_bytes, mask, stream, L))) return st;
+  if ((st = lf_cuda(lf_launch_mask_pass(L), "mask pass"))) return st;
+  return lf_cuda(lf_launch_count(L, counts), "count");
+}
+
+extern "C" int lf_attn_mask_dump(const lf_attn_params *p, const int32_t *mask, uint8_t *out,
+                                 void *workspace, size_t ws_bytes, void *stream) {
+  int st;
+  if (!out) return lf_fail(LF_ERR_INVALID, "out is NULL");
+  LfLaunch L;
+  if ((st = lf_bind_ws(p, 0, workspace, ws_bytes, mask, stream, L))) return st;
+  if (p->n > 8192) return lf_fail(LF_ERR_UNSUPPORTED, "mask dump needs n <= 8192");
+  if ((st = lf_cuda(lf_launch_mask_pass(L), "mask pass"))) return st;
+  return lf_cuda(lf_launch_dump(L, out), "dump");
+}
+
+extern "C" int lf_attn_status(void *workspace, void *stream) {
+  g_err[0] = 0;
+  if (!workspace) return lf_fail(LF_ERR_INVALID, "workspace is NULL");
+  int st;
+  if ((st = lf_cuda(cudaStreamSynchronize((cudaStream_t)stream), "stream sync"))) return st;
+  int32_t w[LF_ST_WORDS];
+  if ((st = lf_cuda(cudaMemcpy(w, workspace, sizeof(w), cudaMemcpyDeviceToHost), "status read")))
+    return st;
+  if ((st = lf_cuda(cudaMemset(workspace, 0, sizeof(w)), "status clear"))) return st;
+  if (w[LF_ST_CODE] == LF_OK) return LF_OK;
+  const int code = w[LF_ST_CODE], det = w[LF_ST_DETAIL];
+  switch (code) {
+    case LF_ERR_DEVICE_INPUT:
+      if (det >= 2000000)
+        return lf_fail(code, "sequence %d has more global tokens than max_global", det - 2000000);
+      return lf_fail(code, "sequence %d has a mask value outside {0,1,2}", det - 1000000);
+    case LF_ERR_UNSUPPORTED:
+      return lf_fail(code, "causal attention with global tokens (sequence %d)", det - 3000000);
+    case LF_ERR_DEVICE_TIMEOUT:
+      return lf_fail(code, "a device-side wait expired (site %d)", det);
+    default: return lf_fail(code, "device status %d (detail %d)", code, det);
+  }
+}

@@ -1,0 +1,447 @@
+// lf_simt.cu -- CUDA-core kernels of the attention library:
+//   * the mask pass (global-token list, valid count, device input checks),
+//   * the pair counter and the pattern dump (tile-walk predicates of the
+//     tensor-core forward),
+//   * the CUDA-core forward and backward for every dtype (the float32 path,
+//     and the cross-check of the tensor-core path for bf16/f16).
+//
+// CUDA-core kernels use one warp per query row (forward, dQ) or per key row
+// (dK, dV); lane l owns head-dim elements 2l and 2l+1, so every K/V/Q row
+// read is one coalesced 128/256-byte access and each score is a warp sum.
+// All sums are float32; outputs are rounded once (RNE) to the call's dtype.
+#include <cub/block/block_scan.cuh>
+
+#include "lf_common.cuh"
+
+// =============================================================== mask pass
+
+// One block per sequence b: compact the global positions (ascending) into
+// gidx[b][0..ng), count valid tokens, flag bad codes, too many globals and
+// causal+global in the status word.
+__global__ void __launch_bounds__(1024) lf_mask_pass_kernel(LfDev P) {
+  typedef cub::BlockScan<int, 1024> Scan;
+  __shared__ typename Scan::TempStorage tmp;
+  __shared__ int s_valid, s_gmin, s_gmax, s_bad, s_total;
+  const int b = blockIdx.x, tid = threadIdx.x, n = P.n;
+  const int32_t *m = P.mask + (size_t)b * n;
+  if (tid == 0) {
+    s_valid = 0;
+    s_gmin = n;
+    s_gmax = -1;
+    s_bad = 0;
+  }
+  __syncthreads();
+  const int per = (n + 1023) / 1024;
+  const int s = tid * per, e = min(n, s + per);
+  int c = 0, v = 0, bad = 0, gmin = n, gmax = -1;
+  for (int i = s; i < e; i++) {
+    int x = m[i];
+    if (x == 2) {
+      c++;
+      gmin = min(gmin, i);
+      gmax = max(gmax, i);
+    }
+    if (x != 0) v++;
+    if (x < 0 || x > 2) bad = 1;
+  }
+  int off, total;
+  Scan(tmp).ExclusiveSum(c, off, total);
+  atomicAdd(&s_valid, v);
+  atomicMin(&s_gmin, gmin);
+  atomicMax(&s_gmax, gmax);
+  if (bad) atomicOr(&s_bad, 1);
+  if (tid == 0) s_total = total;
+  int32_t *gl = P.gidx + (size_t)b * P.G;
+  for (int i = s; i < e && off < P.G; i++)
+    if (m[i] == 2) gl[off++] = i;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t *bi = P.binfo + (size_t)b * LF_BI_WORDS;
+    bi[LF_BI_NG] = min(s_total, P.G);
+    bi[LF_BI_NVALID] = s_valid;
+    bi[LF_BI_GMIN] = s_gmin;
+    bi[LF_BI_GMAX] = s_gmax;
+    if (s_bad) lf_set_status(P.status, LF_ERR_DEVICE_INPUT, 1000000 + b);
+    if (s_total > P.G) lf_set_status(P.status, LF_ERR_DEVICE_INPUT, 2000000 + b);
+    if (P.causal && s_total > 0) lf_set_status(P.status, LF_ERR_UNSUPPORTED, 3000000 + b);
+  }
+}
+
+cudaError_t lf_launch_mask_pass(const LfLaunch &L) {
+  lf_mask_pass_kernel<<<L.dev.B, 1024, 0, L.stream>>>(L.dev);
+  lf_launches_add(1);
+  return cudaGetLastError();
+}
+
+// ===================================================== counter and dump
+
+// Attended keys of row t (sub-sequence coordinates, residue rho, dilation d)
+// enumerated by the tensor-core tile walk: band tiles u = 0.. of the row's
+// 128-row query block, then the global tile minus keys already in the window.
+__device__ int64_t lf_row_pairs_tilewalk(const LfDev &P, int b, int d, int rho, int t) {
+  const int n = P.n, cnt = lf_sub_len(n, d, rho);
+  const int32_t *m = P.mask + (size_t)b * n;
+  const int p = rho + t * d;
+  const int code = m[p];
+  if (code == 0) return 0;
+  const int32_t *bi = P.binfo + (size_t)b * LF_BI_WORDS;
+  if (code == 2) return bi[LF_BI_NVALID];
+  const int t0 = (t / LF_BQ) * LF_BQ, q = t - t0;
+  int64_t c = 0;
+  const int nt = lf_band_tiles(P.r, P.causal);
+  for (int u = 0; u < nt; u++) {
+    int lo, hi;
+    lf_band_cols(q, u, P.r, P.causal, lo, hi);
+    for (int col = lo; col <= hi; col++) {
+      int tk = t0 - P.r + LF_BK * u + col;
+      if (tk >= 0 && tk < cnt && m[rho + tk * d] != 0) c++;
+    }
+  }
+  const int ng = bi[LF_BI_NG];
+  const int32_t *gl = P.gidx + (size_t)b * P.G;
+  for (int g = 0; g < ng; g++)
+    if (!lf_in_window(p, gl[g], P.r, d, P.causal)) c++;
+  return c;
+}
+
+__global__ void __launch_bounds__(256) lf_count_kernel(LfDev P, int64_t *counts) {
+  const int bh = blockIdx.x, h = bh % P.H, b = bh / P.H, d = P.dil[h];
+  int64_t c = 0;
+  for (int p = threadIdx.x; p < P.n; p += blockDim.x) c += lf_row_pairs_tilewalk(P, b, d, p % d, p / d);
+  __shared__ unsigned long long s;
+  if (threadIdx.x == 0) s = 0;
+  __syncthreads();
+  atomicAdd(&s, (unsigned long long)c);
+  __syncthreads();
+  if (threadIdx.x == 0) counts[bh] = (int64_t)s;
+}
+
+cudaError_t lf_launch_count(const LfLaunch &L, int64_t *counts) {
+  lf_count_kernel<<<L.dev.B * L.dev.H, 256, 0, L.stream>>>(L.dev, counts);
+  lf_launches_add(1);
+  return cudaGetLastError();
+}
+
+// One block per (b, h, query position p): row p of the pattern.
+__global__ void __launch_bounds__(256) lf_dump_kernel(LfDev P, uint8_t *out) {
+  const int n = P.n;
+  const int p = blockIdx.x, bh = blockIdx.y, h = bh % P.H, b = bh / P.H, d = P.dil[h];
+  const int32_t *m = P.mask + (size_t)b * n;
+  uint8_t *row = out + ((size_t)bh * n + p) * n;
+  const int code = m[p];
+  const int rho = p % d, t = p / d, t0 = (t / LF_BQ) * LF_BQ, q = t - t0;
+  for (int j = threadIdx.x; j < n; j += blockDim.x) {
+    int a = 0;
+    if (code == 2) {
+      a = m[j] != 0;
+    } else if (code == 1 && m[j] != 0) {
+      int band = 0;
+      if (j % d == rho) {  // same residue: locate key j in the tile walk
+        int tk = j / d;
+        int rel = tk - (t0 - P.r);
+        if (rel >= 0) {
+          int u = rel / LF_BK, col = rel % LF_BK, lo, hi;
+          if (u < lf_band_tiles(P.r, P.causal)) {
+            lf_band_cols(q, u, P.r, P.causal, lo, hi);
+            band = (col >= lo && col <= hi);
+          }
+        }
+      }
+      int glob = (m[j] == 2) && !lf_in_window(p, j, P.r, d, P.causal);
+      a = band | glob;
+    }
+    row[j] = (uint8_t)a;
+  }
+}
+
+cudaError_t lf_launch_dump(const LfLaunch &L, uint8_t *out) {
+  dim3 grid(L.dev.n, L.dev.B * L.dev.H);
+  lf_dump_kernel<<<grid, 256, 0, L.stream>>>(L.dev, out);
+  lf_launches_add(1);
+  return cudaGetLastError();
+}
+
+// ========================================================= CUDA-core fwd
+
+struct LfRowState {
+  float mx, l, a0, a1;
+};
+
+// Online softmax step for key row koff (element offset of lane's pair).
+template <typename T>
+__device__ __forceinline__ void lf_visit(LfRowState &st, float2 q, const T *K, const T *V,
+                                         size_t koff) {
+  float2 k = LfIo<T>::ld2(K + koff);
+  float s = lf_warp_sum(q.x * k.x + q.y * k.y);  // log2 domain (q pre-scaled)
+  float mn = fmaxf(st.mx, s);
+  float al = exp2f(st.mx - mn);
+  float pr = exp2f(s - mn);
+  float2 v = LfIo<T>::ld2(V + koff);
+  st.l = st.l * al + pr;
+  st.a0 = st.a0 * al + pr * v.x;
+  st.a1 = st.a1 * al + pr * v.y;
+  st.mx = mn;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+    lf_simt_fwd_kernel(LfDev P, const T *qs, const T *ks, const T *vs, const T *qg, const T *kg,
+                       const T *vg, T *o, float *lse) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int n = P.n;
+  if (row >= (long long)P.B * P.H * n) return;
+  const int i = (int)(row % n);
+  const int bh = (int)(row / n), h = bh % P.H, b = bh / P.H, d = P.dil[h];
+  const int32_t *m = P.mask + (size_t)b * n;
+  const size_t base = (size_t)bh * n * LF_HD + 2 * lane;
+  const size_t ooff = base + (size_t)i * LF_HD;
+  const int code = m[i];
+  if (code == 0) {
+    LfIo<T>::st2(o + ooff, 0.f, 0.f);
+    if (lse && lane == 0) lse[(size_t)bh * n + i] = -INFINITY;
+    return;
+  }
+  const bool glob = code == 2;
+  const T *Q = glob ? qg : qs, *K = glob ? kg : ks, *V = glob ? vg : vs;
+  float2 q = LfIo<T>::ld2(Q + ooff);
+  q.x *= P.scale_log2;
+  q.y *= P.scale_log2;
+  LfRowState st{-INFINITY, 0.f, 0.f, 0.f};
+  if (glob) {
+    for (int j = 0; j < n; j++)
+      if (m[j] != 0) lf_visit<T>(st, q, K, V, base + (size_t)j * LF_HD);
+  } else {
+    const int khi = P.causal ? 0 : P.r;
+    for (int k = -P.r; k <= khi; k++) {
+      int j = i + k * d;
+      if (j < 0 || j >= n || m[j] == 0) continue;
+      lf_visit<T>(st, q, K, V, base + (size_t)j * LF_HD);
+    }
+    const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
+    const int32_t *gl = P.gidx + (size_t)b * P.G;
+    for (int t = 0; t < ng; t++) {
+      int g = gl[t];
+      if (!lf_in_window(i, g, P.r, d, P.causal)) lf_visit<T>(st, q, K, V, base + (size_t)g * LF_HD);
+    }
+  }
+  const float inv = 1.f / st.l;
+  LfIo<T>::st2(o + ooff, st.a0 * inv, st.a1 * inv);
+  if (lse && lane == 0) lse[(size_t)bh * n + i] = (st.mx + log2f(st.l)) * LF_LN2;
+}
+
+template <typename T>
+static cudaError_t lf_simt_fwd_t(const LfLaunch &L, const void *qs, const void *ks, const void *vs,
+                                 const void *qg, const void *kg, const void *vg, void *o,
+                                 float *lse) {
+  long long rows = (long long)L.dev.B * L.dev.H * L.dev.n;
+  unsigned grid = (unsigned)((rows + 7) / 8);
+  lf_simt_fwd_kernel<T><<<grid, 256, 0, L.stream>>>(
+      L.dev, (const T *)qs, (const T *)ks, (const T *)vs, (const T *)qg, (const T *)kg,
+      (const T *)vg, (T *)o, lse);
+  lf_launches_add(1);
+  return cudaGetLastError();
+}
+
+cudaError_t lf_launch_simt_fwd(const LfLaunch &L, const void *qs, const void *ks, const void *vs,
+                               const void *qg, const void *kg, const void *vg, void *o,
+                               float *lse) {
+  switch (L.dtype) {
+    case LF_F32: return lf_simt_fwd_t<float>(L, qs, ks, vs, qg, kg, vg, o, lse);
+    case LF_BF16: return lf_simt_fwd_t<__nv_bfloat16>(L, qs, ks, vs, qg, kg, vg, o, lse);
+    default: return lf_simt_fwd_t<__half>(L, qs, ks, vs, qg, kg, vg, o, lse);
+  }
+}
+
+// ========================================================= CUDA-core bwd
+
+// delta[row] = sum_c dO[row, c] * O[row, c]   (float32; 0 for mask-0 rows)
+template <typename T>
+__global__ void __launch_bounds__(256)
+    lf_bwd_delta_kernel(LfDev P, const T *o, const T *dO, float *delta) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= (long long)P.B * P.H * P.n) return;
+  const size_t off = (size_t)row * LF_HD + 2 * lane;
+  float2 a = LfIo<T>::ld2(o + off), g = LfIo<T>::ld2(dO + off);
+  float s = lf_warp_sum(a.x * g.x + a.y * g.y);
+  if (lane == 0) delta[row] = s;
+}
+
+// dQ: one warp per query row, same key enumeration as the forward.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    lf_bwd_dq_kernel(LfDev P, const T *qs, const T *ks, const T *vs, const T *qg, const T *kg,
+                     const T *vg, const float *lse, const T *dO, const float *delta, T *dqs,
+                     T *dqg) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int n = P.n;
+  if (row >= (long long)P.B * P.H * n) return;
+  const int i = (int)(row % n);
+  const int bh = (int)(row / n), h = bh % P.H, b = bh / P.H, d = P.dil[h];
+  const int32_t *m = P.mask + (size_t)b * n;
+  const size_t base = (size_t)bh * n * LF_HD + 2 * lane;
+  const size_t ioff = base + (size_t)i * LF_HD;
+  const int code = m[i];
+  if (code != 1) LfIo<T>::st2(dqs + ioff, 0.f, 0.f);
+  if (code != 2) LfIo<T>::st2(dqg + ioff, 0.f, 0.f);
+  if (code == 0) return;
+  const bool glob = code == 2;
+  const T *Q = glob ? qg : qs, *K = glob ? kg : ks, *V = glob ? vg : vs;
+  float2 q = LfIo<T>::ld2(Q + ioff);
+  float2 g = LfIo<T>::ld2(dO + ioff);
+  const float L2 = lse[row] * LF_LOG2E, Di = delta[row];
+  float acc0 = 0.f, acc1 = 0.f;
+  auto visit = [&](int j) {
+    size_t koff = base + (size_t)j * LF_HD;
+    float2 k = LfIo<T>::ld2(K + koff), v = LfIo<T>::ld2(V + koff);
+    float2 sd = lf_warp_sum2(q.x * k.x + q.y * k.y, g.x * v.x + g.y * v.y);
+    float pr = exp2f(sd.x * P.scale_log2 - L2);
+    float ds = pr * (sd.y - Di) * P.scale;
+    acc0 += ds * k.x;
+    acc1 += ds * k.y;
+  };
+  if (glob) {
+    for (int j = 0; j < n; j++)
+      if (m[j] != 0) visit(j);
+  } else {
+    const int khi = P.causal ? 0 : P.r;
+    for (int k = -P.r; k <= khi; k++) {
+      int j = i + k * d;
+      if (j < 0 || j >= n || m[j] == 0) continue;
+      visit(j);
+    }
+    const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
+    const int32_t *gl = P.gidx + (size_t)b * P.G;
+    for (int t = 0; t < ng; t++)
+      if (!lf_in_window(i, gl[t], P.r, d, P.causal)) visit(gl[t]);
+  }
+  LfIo<T>::st2((glob ? dqg : dqs) + ioff, acc0, acc1);
+}
+
+// dK_s, dV_s: one warp per key row j, over the LOCAL rows that attend j.
+// A non-global key is attended by the rows i = j - k*d of its window; a
+// global key by every local row (exactly once: window or global column).
+template <typename T>
+__global__ void __launch_bounds__(256)
+    lf_bwd_dkv_s_kernel(LfDev P, const T *qs, const T *ks, const T *vs, const float *lse,
+                        const T *dO, const float *delta, T *dks, T *dvs) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int n = P.n;
+  if (row >= (long long)P.B * P.H * n) return;
+  const int j = (int)(row % n);
+  const int bh = (int)(row / n), h = bh % P.H, b = bh / P.H, d = P.dil[h];
+  const int32_t *m = P.mask + (size_t)b * n;
+  const size_t base = (size_t)bh * n * LF_HD + 2 * lane;
+  const size_t joff = base + (size_t)j * LF_HD;
+  const int code = m[j];
+  float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+  if (code != 0) {
+    float2 kk = LfIo<T>::ld2(ks + joff), vv = LfIo<T>::ld2(vs + joff);
+    auto visit = [&](int i) {
+      size_t ioff = base + (size_t)i * LF_HD;
+      size_t ir = (size_t)bh * n + i;
+      float2 q = LfIo<T>::ld2(qs + ioff), g = LfIo<T>::ld2(dO + ioff);
+      float2 sd = lf_warp_sum2(q.x * kk.x + q.y * kk.y, g.x * vv.x + g.y * vv.y);
+      float pr = exp2f(sd.x * P.scale_log2 - lse[ir] * LF_LOG2E);
+      float ds = pr * (sd.y - delta[ir]) * P.scale;
+      k0 += ds * q.x;
+      k1 += ds * q.y;
+      v0 += pr * g.x;
+      v1 += pr * g.y;
+    };
+    if (code == 2) {
+      for (int i = 0; i < n; i++)
+        if (m[i] == 1) visit(i);
+    } else {
+      // row i attends j when j = i + k*d with k in [-r, khi]  <=>  i = j - k*d
+      const int khi = P.causal ? 0 : P.r;
+      for (int k = khi; k >= -P.r; k--) {
+        int i = j - k * d;
+        if (i < 0 || i >= n || m[i] != 1) continue;
+        visit(i);
+      }
+    }
+  }
+  LfIo<T>::st2(dks + joff, k0, k1);
+  LfIo<T>::st2(dvs + joff, v0, v1);
+}
+
+// dK_g, dV_g: one warp per key row j, over the global rows (every global
+// row attends every valid key through Q_g / K_g / V_g).
+template <typename T>
+__global__ void __launch_bounds__(256)
+    lf_bwd_dkv_g_kernel(LfDev P, const T *qg, const T *kg, const T *vg, const float *lse,
+                        const T *dO, const float *delta, T *dkg, T *dvg) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int n = P.n;
+  if (row >= (long long)P.B * P.H * n) return;
+  const int j = (int)(row % n);
+  const int bh = (int)(row / n), b = bh / P.H;
+  const int32_t *m = P.mask + (size_t)b * n;
+  const size_t base = (size_t)bh * n * LF_HD + 2 * lane;
+  const size_t joff = base + (size_t)j * LF_HD;
+  float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+  if (m[j] != 0) {
+    float2 kk = LfIo<T>::ld2(kg + joff), vv = LfIo<T>::ld2(vg + joff);
+    const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
+    const int32_t *gl = P.gidx + (size_t)b * P.G;
+    for (int t = 0; t < ng; t++) {
+      int i = gl[t];
+      size_t ioff = base + (size_t)i * LF_HD;
+      size_t ir = (size_t)bh * n + i;
+      float2 q = LfIo<T>::ld2(qg + ioff), g = LfIo<T>::ld2(dO + ioff);
+      float2 sd = lf_warp_sum2(q.x * kk.x + q.y * kk.y, g.x * vv.x + g.y * vv.y);
+      float pr = exp2f(sd.x * P.scale_log2 - lse[ir] * LF_LOG2E);
+      float ds = pr * (sd.y - delta[ir]) * P.scale;
+      k0 += ds * q.x;
+      k1 += ds * q.y;
+      v0 += pr * g.x;
+      v1 += pr * g.y;
+    }
+  }
+  LfIo<T>::st2(dkg + joff, k0, k1);
+  LfIo<T>::st2(dvg + joff, v0, v1);
+}
+
+template <typename T>
+static cudaError_t lf_simt_bwd_t(const LfLaunch &L, const void *qs, const void *ks, const void *vs,
+                                 const void *qg, const void *kg, const void *vg, const void *o,
+                                 const float *lse, const void *dO, void *dqs, void *dks, void *dvs,
+                                 void *dqg, void *dkg, void *dvg) {
+  long long rows = (long long)L.dev.B * L.dev.H * L.dev.n;
+  unsigned grid = (unsigned)((rows + 7) / 8);
+  float *delta = (float *)(L.ws_base + L.ws.delta);
+  lf_bwd_delta_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)o, (const T *)dO, delta);
+  lf_bwd_dq_kernel<T><<<grid, 256, 0, L.stream>>>(
+      L.dev, (const T *)qs, (const T *)ks, (const T *)vs, (const T *)qg, (const T *)kg,
+      (const T *)vg, lse, (const T *)dO, delta, (T *)dqs, (T *)dqg);
+  lf_bwd_dkv_s_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)qs, (const T *)ks,
+                                                     (const T *)vs, lse, (const T *)dO, delta,
+                                                     (T *)dks, (T *)dvs);
+  lf_bwd_dkv_g_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)qg, (const T *)kg,
+                                                     (const T *)vg, lse, (const T *)dO, delta,
+                                                     (T *)dkg, (T *)dvg);
+  lf_launches_add(4);
+  return cudaGetLastError();
+}
+
+cudaError_t lf_launch_simt_bwd(const LfLaunch &L, const void *qs, const void *ks, const void *vs,
+                               const void *qg, const void *kg, const void *vg, const void *o,
+                               const float *lse, const void *dO, void *dqs, void *dks, void *dvs,
+                               void *dqg, void *dkg, void *dvg) {
+  switch (L.dtype) {
+    case LF_F32:
+      return lf_simt_bwd_t<float>(L, qs, ks, vs, qg, kg, vg, o, lse, dO, dqs, dks, dvs, dqg, dkg,
+                                  dvg);
+    case LF_BF16:
+      return lf_simt_bwd_t<__nv_bfloat16>(L, qs, ks, vs, qg, kg, vg, o, lse, dO, dqs, dks, dvs,
+                                          dqg, dkg, dvg);
+    default:
+      return lf_simt_bwd_t<__half>(L, qs, ks, vs, qg, kg, vg, o, lse, dO, dqs, dks, dvs, dqg,
+                                   dkg, dvg);
+  }
+}

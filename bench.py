@@ -269,6 +269,9 @@ def main():
     # kernel timing events (main attention kernel of every timed step)
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
+    for a, b in kev:  # create the CUDA events; the library re-records them
+        a.record(stream)
+        b.record(stream)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()

@@ -177,6 +177,15 @@ extern "C" int lf_attn_fwd(const lf_attn_params *p, const void *q_s, const void 
   if (tc) {
     LfTcArgs a{q_s, k_s, v_s, q_g, k_g, v_g, o, lse, g_ev_start, g_ev_stop};
     st = lf_tc_fwd(L, a, g_err, sizeof(g_err));
+    if (st == LF_ERR_UNSUPPORTED && p->kernel == LF_KERNEL_AUTO) {
+      // shape outside the tensor-core kernel's parameter block: CUDA-core kernel
+      g_err[0] = 0;
+      st = LF_OK;
+      if (g_ev_start && g_ev_stop) cudaEventRecord(g_ev_start, L.stream);
+      if ((st = lf_cuda(lf_launch_simt_fwd(L, q_s, k_s, v_s, q_g, k_g, v_g, o, lse), "forward")))
+        return st;
+      if (g_ev_start && g_ev_stop) cudaEventRecord(g_ev_stop, L.stream);
+    }
     if (st) return st;
   } else {
     if (g_ev_start && g_ev_stop) cudaEventRecord(g_ev_start, L.stream);

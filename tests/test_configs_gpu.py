@@ -29,8 +29,11 @@ def _run(name):
     wl = synth.WORKLOADS[name]
     inp = synth.make_inputs(wl)
     ng = int((inp["mask"] == 2).sum(axis=1).max())
+    # bench.py's default selection: tensor cores for bf16/f16 (requested
+    # explicitly here so a silent CUDA-core fallback would fail the test)
+    kern = L.LF_KERNEL_SIMT if wl.dtype == "f32" else L.LF_KERNEL_TC
     att = L.LongformerAttention(wl.B, wl.H, wl.n, wl.r, wl.dilation, wl.causal, dtype=wl.dtype,
-                                max_global=ng)
+                                max_global=ng, kernel=kern)
     g = U.gpu_inputs(inp, wl.dtype)
     o, lse = att.fwd(g["qs"], g["ks"], g["vs"], g["qg"], g["kg"], g["vg"], g["mask"])
     att.status()

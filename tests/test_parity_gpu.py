@@ -61,7 +61,7 @@ def _cases():
 
 CASES = _cases()
 KERNELS = [("f32", L.LF_KERNEL_SIMT), ("bf16", L.LF_KERNEL_SIMT), ("f16", L.LF_KERNEL_SIMT),
-           ("bf16", L.LF_KERNEL_AUTO), ("f16", L.LF_KERNEL_AUTO)]
+           ("bf16", L.LF_KERNEL_TC), ("f16", L.LF_KERNEL_TC), ("f32", L.LF_KERNEL_AUTO)]
 
 
 def _setup(name, dtype, kernel, seed=11, backward=False):

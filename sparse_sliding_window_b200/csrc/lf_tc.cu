@@ -292,6 +292,60 @@ __device__ __forceinline__ uint32_t lf_idesc(int f16, int n, int b_mn) {
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
+// Bits k (0..31) of the 32-column chunk starting at column `base` whose
+// column lies in [lo, hi].
+__device__ __forceinline__ uint32_t lf_range_bits(int lo, int hi, int base) {
+  int a = lo - base, z = hi - base;
+  if (z < 0 || a > 31 || a > z) return 0u;
+  a = max(a, 0);
+  z = min(z, 31);
+  const uint32_t upto = z == 31 ? 0xffffffffu : ((1u << (z + 1)) - 1u);
+  return upto & ~((1u << a) - 1u);
+}
+
+// One pass over the 4 column chunks of a row's S tile (TMEM lane of this
+// thread).  Columns whose bit in w is clear are treated as -inf.  Tracks the
+// row max of the attended raw scores in mx; when write_p, also computes
+// p = 2^(s * sl2 - m) into P (TMEM, packed bf16 / f16) and their sum lt.
+// Chunks no lane of the warp attends are skipped (P written as zeros).
+template <int kF16>
+__device__ __forceinline__ void lf_softmax_tile(uint32_t tl, const uint32_t (&w)[4], float sl2,
+                                                float m, float &mx, float &lt, bool write_p) {
+  const float mneg = m == -INFINITY ? 0.f : -m;
+#pragma unroll
+  for (int cc = 0; cc < 4; cc++) {
+    const uint32_t wc = w[cc];
+    if (!__any_sync(0xffffffffu, wc != 0u)) {
+      if (write_p) {
+        uint32_t z[16];
+#pragma unroll
+        for (int k = 0; k < 16; k++) z[k] = 0u;
+        lf_tmem_st16(tl + LF_TM_P + 16 * cc, z);
+      }
+      continue;
+    }
+    float x[32];
+    lf_tmem_ld32(tl + LF_TM_S + 32 * cc, x);
+    if (!__all_sync(0xffffffffu, wc == 0xffffffffu)) {
+#pragma unroll
+      for (int k = 0; k < 32; k++) x[k] = ((wc >> k) & 1u) ? x[k] : -INFINITY;
+    }
+#pragma unroll
+    for (int k = 0; k < 32; k++) mx = fmaxf(mx, x[k]);
+    if (write_p) {
+      uint32_t pw[16];
+#pragma unroll
+      for (int k = 0; k < 32; k += 2) {
+        const float p0 = lf_ex2(fmaf(x[k], sl2, mneg));
+        const float p1 = lf_ex2(fmaf(x[k + 1], sl2, mneg));
+        lt += p0 + p1;
+        pw[k / 2] = lf_pack2<kF16>(p0, p1);
+      }
+      lf_tmem_st16(tl + LF_TM_P + 16 * cc, pw);
+    }
+  }
+}
+
 // ------------------------------------------------------------ the kernel
 
 template <int kF16>
@@ -497,6 +551,26 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 2)
     }
     const int32_t *gl = D.gidx + (size_t)b * D.G;
     const float sl2 = D.scale_log2;
+    const bool padded = D.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NVALID] < n;
+    // Global keys already in this row's window: positions [pos - r d, pos + r d]
+    // (causal: up to pos) of the row's residue.  gidx is sorted, so they form
+    // the index range [e_lo, e_hi) filtered by residue.
+    int e_lo = 0, e_hi = 0;
+    if (!gitem && nglob > 0 && active) {
+      const int lo_pos = pos - D.r * d, hi_pos = D.causal ? pos : pos + D.r * d;
+      int a = 0, z = ng;
+      while (a < z) {  // first e with gl[e] >= lo_pos
+        const int mid = (a + z) >> 1;
+        if (gl[mid] < lo_pos) a = mid + 1; else z = mid;
+      }
+      e_lo = a;
+      z = ng;
+      while (a < z) {  // first e with gl[e] > hi_pos
+        const int mid = (a + z) >> 1;
+        if (gl[mid] <= hi_pos) a = mid + 1; else z = mid;
+      }
+      e_hi = a;
+    }
     float m_ref = -INFINITY, l = 0.f;
     bool alive = true;
     for (int it = 0; it < T && alive; it++) {
@@ -505,95 +579,73 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 2)
         break;
       }
       lf_tc_fence_after();
-      // ---- which columns of this tile may row q attend
-      uint32_t vw[4];
-      int lo = 0, hi = LF_BK - 1, nch = 4;
-      bool gtile = !gitem && it >= nband;
-      int gtl_base = 0;
-      if (!gtile) {
+      // ---- attend mask of row q over the tile's 128 columns (4 words)
+      uint32_t w[4];
+      if (it < nband) {
         const int kb = gitem ? (kt0 + it) * LF_BK : tk0 + it * LF_BK;
+        int lo = 0, hi = LF_BK - 1;
+        if (!gitem) lf_band_cols(q, it, D.r, D.causal, lo, hi);
+        lo = max(lo, -kb);            // keys exist on [0, cnt)
+        hi = min(hi, cnt - 1 - kb);
+        if (!active) hi = -1;
+#pragma unroll
+        for (int cc = 0; cc < 4; cc++) w[cc] = lf_range_bits(lo, hi, 32 * cc);
+        if (padded) {
+#pragma unroll
+          for (int cc = 0; cc < 4; cc++) {
+            const int tk = kb + 32 * cc + lane;
+            const bool ok = tk >= 0 && tk < cnt && mrow[rho + tk * d] != 0;
+            w[cc] &= __ballot_sync(0xffffffffu, ok);
+          }
+        }
+      } else {
+        const int gb = (it - nband) * LF_BK;
+        const int hi = active ? min(LF_BK - 1, ng - 1 - gb) : -1;
 #pragma unroll
         for (int cc = 0; cc < 4; cc++) {
-          const int tk = kb + 32 * cc + lane;
-          bool ok = tk >= 0 && tk < cnt && mrow[rho + tk * d] != 0;
-          vw[cc] = __ballot_sync(0xffffffffu, ok);
+          uint32_t inwin = lf_range_bits(e_lo - gb, e_hi - 1 - gb, 32 * cc);
+          if (d > 1) {
+            const int e = gb + 32 * cc + lane;
+            const bool res = e < ng && (gl[e] - rho) % d == 0;
+            inwin &= __ballot_sync(0xffffffffu, res);
+          }
+          w[cc] = lf_range_bits(0, hi, 32 * cc) & ~inwin;
         }
-        if (!gitem) lf_band_cols(q, it, D.r, D.causal, lo, hi);
-      } else {
-        gtl_base = (it - nband) * LF_BK;
-        const int ngk = (ng + 15) / 16 * 16;
-        nch = (min(LF_BK, ngk - gtl_base) + 31) / 32;
-#pragma unroll
-        for (int cc = 0; cc < 4; cc++) vw[cc] = 0;  // per-row bits are built below
       }
-      // ---- pass 1: row max over attended columns
-      float mt = -INFINITY;
-      for (int cc = 0; cc < nch; cc++) {
-        float x[32];
-        lf_tmem_ld32(tl + LF_TM_S + 32 * cc, x);
-        uint32_t g_own = 0;
-        if (gtile) {
-          // bit k set when column 32cc+k is attended by THIS row
-          const int e0 = gtl_base + 32 * cc;
-          const int myg = (e0 + lane < ng) ? gl[e0 + lane] : -1;
+      // ---- probabilities of the tile -> P (TMEM).  Optimistic single pass
+      // against the running reference m_ref; redone (rarely) with the tile's
+      // own max when some row's max grew by more than 2^8.
+      const bool any_bits = (w[0] | w[1] | w[2] | w[3]) != 0u;
+      const bool single = __all_sync(0xffffffffu, m_ref != -INFINITY || !any_bits);
+      float mx = -INFINITY, lt = 0.f;
+      if (single) lf_softmax_tile<kF16>(tl, w, sl2, m_ref, mx, lt, true);
+      const bool grow = any_bits && (!single || mx * sl2 > m_ref + 8.f);
+      if (__any_sync(0xffffffffu, grow)) {
+        if (!single) {
+          float dummy = 0.f;
+          lf_softmax_tile<kF16>(tl, w, sl2, m_ref, mx, dummy, false);  // max only
+        }
+        const float ms = mx * sl2;
+        const bool need = any_bits && ms > m_ref + 8.f;
+        const float m_new = need ? ms : m_ref;
+        const float alpha = need ? lf_ex2(m_ref - m_new) : 1.f;
+        l *= alpha;
+        if (it > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
-          for (int k = 0; k < 32; k++) {
-            const int g = __shfl_sync(0xffffffffu, myg, k);
-            if (g >= 0 && !lf_in_window(pos, g, D.r, d, D.causal)) g_own |= 1u << k;
+          for (int half = 0; half < 2; half++) {
+            float ov[32];
+            lf_tmem_ld32(tl + LF_TM_O + 32 * half, ov);
+#pragma unroll
+            for (int k = 0; k < 32; k++) ov[k] *= alpha;
+            lf_tmem_st32(tl + LF_TM_O + 32 * half, ov);
           }
         }
-        const uint32_t w = gtile ? g_own : vw[cc];
-#pragma unroll
-        for (int k = 0; k < 32; k++) {
-          const int c = 32 * cc + k;
-          const bool ok = active && ((w >> k) & 1u) && c >= lo && c <= hi;
-          if (ok) mt = fmaxf(mt, x[k]);
-        }
+        m_ref = m_new;
+        lt = 0.f;
+        float mx2 = -INFINITY;
+        lf_softmax_tile<kF16>(tl, w, sl2, m_ref, mx2, lt, true);
       }
-      mt *= sl2;
-      const bool need = mt > m_ref + 8.f;
-      const float m_new = need ? mt : m_ref;
-      const float alpha = need ? lf_ex2(m_ref - m_new) : 1.f;
-      l *= alpha;
-      if (it > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
-        for (int half = 0; half < 2; half++) {
-          float ov[32];
-          lf_tmem_ld32(tl + LF_TM_O + 32 * half, ov);
-#pragma unroll
-          for (int k = 0; k < 32; k++) ov[k] *= alpha;
-          lf_tmem_st32(tl + LF_TM_O + 32 * half, ov);
-        }
-      }
-      m_ref = m_new;
-      // ---- pass 2: probabilities -> P (TMEM), row sum
-      for (int cc = 0; cc < nch; cc++) {
-        float x[32];
-        lf_tmem_ld32(tl + LF_TM_S + 32 * cc, x);
-        uint32_t w = vw[cc];
-        if (gtile) {
-          const int e0 = gtl_base + 32 * cc;
-          const int myg = (e0 + lane < ng) ? gl[e0 + lane] : -1;
-          w = 0;
-#pragma unroll
-          for (int k = 0; k < 32; k++) {
-            const int g = __shfl_sync(0xffffffffu, myg, k);
-            if (g >= 0 && !lf_in_window(pos, g, D.r, d, D.causal)) w |= 1u << k;
-          }
-        }
-        uint32_t pw[16];
-#pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          const int c = 32 * cc + k;
-          const bool ok0 = active && ((w >> k) & 1u) && c >= lo && c <= hi;
-          const bool ok1 = active && ((w >> (k + 1)) & 1u) && c + 1 >= lo && c + 1 <= hi;
-          const float p0 = ok0 ? lf_ex2(fmaf(x[k], sl2, -m_ref)) : 0.f;
-          const float p1 = ok1 ? lf_ex2(fmaf(x[k + 1], sl2, -m_ref)) : 0.f;
-          l += p0 + p1;
-          pw[k / 2] = lf_pack2<kF16>(p0, p1);
-        }
-        lf_tmem_st16(tl + LF_TM_P + 16 * cc, pw);
-      }
+      l += lt;
       lf_tmem_wait_st();
       lf_tc_fence_before();
       __syncwarp();

@@ -104,6 +104,8 @@ static int lf_prepare(const lf_attn_params *p, int for_bwd, LfDev &dev, LfWs &ws
   off = lf_align(off + B * LF_BI_WORDS * 4);
   ws.gidx = off;
   off = lf_align(off + B * Ga * 4);
+  ws.grank = off;
+  off = lf_align(off + B * ((size_t)n + 1) * 4);
   const bool tc = p->dtype != LF_F32 && p->kernel != LF_KERNEL_SIMT;
   ws.qg_c = ws.ks_c = ws.vs_c = ws.part_acc = ws.part_ml = off;
   if (tc && !for_bwd) {
@@ -156,6 +158,7 @@ static int lf_bind_ws(const lf_attn_params *p, int for_bwd, void *workspace, siz
   L.dev.status = (int32_t *)(L.ws_base + L.ws.status);
   L.dev.binfo = (int32_t *)(L.ws_base + L.ws.binfo);
   L.dev.gidx = (int32_t *)(L.ws_base + L.ws.gidx);
+  L.dev.grank = (int32_t *)(L.ws_base + L.ws.grank);
   // each call starts with a clear status word; lf_attn_status reads it back
   return lf_cuda(cudaMemsetAsync(L.dev.status, 0, LF_ST_WORDS * 4, L.stream), "status reset");
 }

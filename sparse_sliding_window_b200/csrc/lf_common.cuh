@@ -34,6 +34,7 @@ struct LfWs {
   size_t status;    // int32[LF_ST_WORDS]
   size_t binfo;     // int32[B][LF_BI_WORDS]
   size_t gidx;      // int32[B][G]           global positions, ascending
+  size_t grank;     // int32[B][n+1]         globals at positions < p
   size_t qg_c;      // T[B][H][G][64]        Q_g rows of the global tokens
   size_t ks_c;      // T[B][H][Gk][64]       K_s rows of the global tokens (zero padded)
   size_t vs_c;      // T[B][H][Gk][64]       V_s rows of the global tokens (zero padded)
@@ -55,6 +56,7 @@ struct LfDev {
   int32_t *status;
   int32_t *binfo;
   int32_t *gidx;
+  int32_t *grank;
   int dil[LF_MAX_H];
 };
 

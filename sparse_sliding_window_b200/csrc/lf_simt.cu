@@ -16,7 +16,8 @@
 // =============================================================== mask pass
 
 // One block per sequence b: compact the global positions (ascending) into
-// gidx[b][0..ng), count valid tokens, flag bad codes, too many globals and
+// gidx[b][0..ng), write the rank array grank[b][p] = #globals before p,
+// count valid tokens, flag bad codes, too many globals and
 // causal+global in the status word.
 __global__ void __launch_bounds__(1024) lf_mask_pass_kernel(LfDev P) {
   typedef cub::BlockScan<int, 1024> Scan;
@@ -52,8 +53,15 @@ __global__ void __launch_bounds__(1024) lf_mask_pass_kernel(LfDev P) {
   if (bad) atomicOr(&s_bad, 1);
   if (tid == 0) s_total = total;
   int32_t *gl = P.gidx + (size_t)b * P.G;
-  for (int i = s; i < e && off < P.G; i++)
-    if (m[i] == 2) gl[off++] = i;
+  int32_t *gr = P.grank + (size_t)b * (n + 1);
+  for (int i = s; i < e; i++) {
+    gr[i] = off;  // globals before position i
+    if (m[i] == 2) {
+      if (off < P.G) gl[off] = i;
+      off++;
+    }
+  }
+  if (tid == 1023) gr[n] = total;
   __syncthreads();
   if (tid == 0) {
     int32_t *bi = P.binfo + (size_t)b * LF_BI_WORDS;

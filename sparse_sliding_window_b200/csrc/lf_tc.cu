@@ -52,7 +52,7 @@
 #include "lf_tc.cuh"
 
 #define LF_TC_THREADS 192
-#define LF_TC_NS 2
+#define LF_TC_NS 3
 #define LF_TC_MAX_MAPS 28
 #define LF_TC_MAX_SEG 32
 #define LF_WAIT_NS 1500000000ull
@@ -68,7 +68,7 @@
 #define LF_SM_K(s) (16384 + (s)*16384)
 #define LF_SM_V(s) (16384 + LF_TC_NS * 16384 + (s)*16384)
 #define LF_SM_BAR (16384 + 2 * LF_TC_NS * 16384)
-#define LF_SMEM_BYTES (1024 + LF_SM_BAR + 256)
+#define LF_SMEM_BYTES (LF_SM_BAR + 256)
 
 struct LfTcSeg {
   int h0, h1, d, rho, cnt, nqb, start, map;
@@ -309,39 +309,113 @@ __device__ __forceinline__ uint32_t lf_range_bits(int lo, int hi, int base) {
 // p = 2^(s * sl2 - m) into P (TMEM, packed bf16 / f16) and their sum lt.
 // Chunks no lane of the warp attends are skipped (P written as zeros).
 template <int kF16>
+__device__ __forceinline__ void lf_p_chunk(uint32_t tl, int cc, float (&x)[32], float sl2,
+                                           float mneg, float &lt) {
+  uint32_t pw[16];
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 32; k += 2) {
+    const float p0 = lf_ex2(fmaf(x[k], sl2, mneg));
+    const float p1 = lf_ex2(fmaf(x[k + 1], sl2, mneg));
+    s0 += p0;
+    s1 += p1;
+    pw[k / 2] = lf_pack2<kF16>(p0, p1);
+  }
+  lt += s0 + s1;
+  lf_tmem_st16(tl + LF_TM_P + 16 * cc, pw);
+}
+
+__device__ __forceinline__ void lf_mask_chunk(float (&x)[32], uint32_t wc) {
+  if (!__all_sync(0xffffffffu, wc == 0xffffffffu)) {
+#pragma unroll
+    for (int k = 0; k < 32; k++) x[k] = ((wc >> k) & 1u) ? x[k] : -INFINITY;
+  }
+}
+
+__device__ __forceinline__ float lf_max32(const float (&x)[32]) {
+  float a = fmaxf(x[0], x[1]), b = fmaxf(x[2], x[3]), c = fmaxf(x[4], x[5]), d = fmaxf(x[6], x[7]);
+#pragma unroll
+  for (int k = 8; k < 32; k += 4) {
+    a = fmaxf(a, x[k]);
+    b = fmaxf(b, x[k + 1]);
+    c = fmaxf(c, x[k + 2]);
+    d = fmaxf(d, x[k + 3]);
+  }
+  return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
+// 64 consecutive fp32 columns of this thread's TMEM lane (one wait)
+__device__ __forceinline__ void lf_tmem_ld32x2(uint32_t taddr, float (&x)[32], float (&y)[32]) {
+  uint32_t r[32], u[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+        "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]),
+        "=r"(u[13]), "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]),
+        "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]),
+        "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]),
+        "=r"(u[31])
+      : "r"(taddr + 32));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int k = 0; k < 32; k++) {
+    x[k] = __uint_as_float(r[k]);
+    y[k] = __uint_as_float(u[k]);
+  }
+}
+
+// One pass over the 4 column chunks of a row's S tile (TMEM lane of this
+// thread).  Columns whose bit in w is clear are treated as -inf.  Tracks the
+// row max of the attended raw scores in mx; when write_p, also computes
+// p = 2^(s * sl2 - m) into P (TMEM, packed bf16 / f16) and their sum lt.
+// Chunks no lane of the warp attends are skipped (P written as zeros); two
+// attended chunks are fetched with one TMEM wait.
+template <int kF16>
 __device__ __forceinline__ void lf_softmax_tile(uint32_t tl, const uint32_t (&w)[4], float sl2,
                                                 float m, float &mx, float &lt, bool write_p) {
   const float mneg = m == -INFINITY ? 0.f : -m;
 #pragma unroll
-  for (int cc = 0; cc < 4; cc++) {
-    const uint32_t wc = w[cc];
-    if (!__any_sync(0xffffffffu, wc != 0u)) {
+  for (int pp = 0; pp < 2; pp++) {
+    const int c0 = 2 * pp, c1 = 2 * pp + 1;
+    const bool a0 = __any_sync(0xffffffffu, w[c0] != 0u);
+    const bool a1 = __any_sync(0xffffffffu, w[c1] != 0u);
+    if (write_p && !(a0 && a1)) {
+      uint32_t z[16];
+#pragma unroll
+      for (int k = 0; k < 16; k++) z[k] = 0u;
+      if (!a0) lf_tmem_st16(tl + LF_TM_P + 16 * c0, z);
+      if (!a1) lf_tmem_st16(tl + LF_TM_P + 16 * c1, z);
+    }
+    if (a0 && a1) {
+      float x[32], y[32];
+      lf_tmem_ld32x2(tl + LF_TM_S + 32 * c0, x, y);
+      lf_mask_chunk(x, w[c0]);
+      lf_mask_chunk(y, w[c1]);
+      mx = fmaxf(mx, fmaxf(lf_max32(x), lf_max32(y)));
       if (write_p) {
-        uint32_t z[16];
-#pragma unroll
-        for (int k = 0; k < 16; k++) z[k] = 0u;
-        lf_tmem_st16(tl + LF_TM_P + 16 * cc, z);
+        lf_p_chunk<kF16>(tl, c0, x, sl2, mneg, lt);
+        lf_p_chunk<kF16>(tl, c1, y, sl2, mneg, lt);
       }
-      continue;
-    }
-    float x[32];
-    lf_tmem_ld32(tl + LF_TM_S + 32 * cc, x);
-    if (!__all_sync(0xffffffffu, wc == 0xffffffffu)) {
-#pragma unroll
-      for (int k = 0; k < 32; k++) x[k] = ((wc >> k) & 1u) ? x[k] : -INFINITY;
-    }
-#pragma unroll
-    for (int k = 0; k < 32; k++) mx = fmaxf(mx, x[k]);
-    if (write_p) {
-      uint32_t pw[16];
-#pragma unroll
-      for (int k = 0; k < 32; k += 2) {
-        const float p0 = lf_ex2(fmaf(x[k], sl2, mneg));
-        const float p1 = lf_ex2(fmaf(x[k + 1], sl2, mneg));
-        lt += p0 + p1;
-        pw[k / 2] = lf_pack2<kF16>(p0, p1);
-      }
-      lf_tmem_st16(tl + LF_TM_P + 16 * cc, pw);
+    } else if (a0 || a1) {
+      const int c = a0 ? c0 : c1;
+      float x[32];
+      lf_tmem_ld32(tl + LF_TM_S + 32 * c, x);
+      lf_mask_chunk(x, w[c]);
+      mx = fmaxf(mx, lf_max32(x));
+      if (write_p) lf_p_chunk<kF16>(tl, c, x, sl2, mneg, lt);
     }
   }
 }
@@ -351,10 +425,15 @@ __device__ __forceinline__ void lf_softmax_tile(uint32_t tl, const uint32_t (&w)
 template <int kF16>
 __global__ void __launch_bounds__(LF_TC_THREADS, 2)
     lf_tc_fwd_kernel(const __grid_constant__ LfTcParams P) {
-  extern __shared__ uint8_t lf_smem_raw[];
-  const uint32_t raw = lf_smem(lf_smem_raw);
-  const uint32_t sbase = (raw + 1023u) & ~1023u;
-  uint8_t *gbase = lf_smem_raw + (sbase - raw);
+  extern __shared__ __align__(1024) uint8_t lf_smem_raw[];
+  // the dynamic shared window starts 1024-byte aligned (128-byte swizzled
+  // TMA tiles need it); checked rather than padded, to fit two CTAs per SM
+  const uint32_t sbase = lf_smem(lf_smem_raw);
+  uint8_t *gbase = lf_smem_raw;
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) lf_set_status(P.dev.status, LF_ERR_UNSUPPORTED, 9000);
+    return;
+  }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const LfDev &D = P.dev;
@@ -554,22 +633,15 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 2)
     const bool padded = D.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NVALID] < n;
     // Global keys already in this row's window: positions [pos - r d, pos + r d]
     // (causal: up to pos) of the row's residue.  gidx is sorted, so they form
-    // the index range [e_lo, e_hi) filtered by residue.
+    // the index range [e_lo, e_hi) = [rank(pos - r d), rank(pos + r d + 1)),
+    // filtered by residue.
     int e_lo = 0, e_hi = 0;
     if (!gitem && nglob > 0 && active) {
-      const int lo_pos = pos - D.r * d, hi_pos = D.causal ? pos : pos + D.r * d;
-      int a = 0, z = ng;
-      while (a < z) {  // first e with gl[e] >= lo_pos
-        const int mid = (a + z) >> 1;
-        if (gl[mid] < lo_pos) a = mid + 1; else z = mid;
-      }
-      e_lo = a;
-      z = ng;
-      while (a < z) {  // first e with gl[e] > hi_pos
-        const int mid = (a + z) >> 1;
-        if (gl[mid] <= hi_pos) a = mid + 1; else z = mid;
-      }
-      e_hi = a;
+      const int32_t *gr = D.grank + (size_t)b * (n + 1);
+      const int lo_pos = max(pos - D.r * d, 0);
+      const int hi_pos = min((D.causal ? pos : pos + D.r * d) + 1, n);
+      e_lo = gr[lo_pos];
+      e_hi = gr[hi_pos];
     }
     float m_ref = -INFINITY, l = 0.f;
     bool alive = true;

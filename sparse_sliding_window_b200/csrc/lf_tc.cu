@@ -145,20 +145,20 @@ __device__ __noinline__ bool lf_wait(uint32_t bar, uint32_t parity, volatile int
   }
 }
 
-// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast, then
-// every lane observes the completed phase itself (acquire) before the
+// Bounded wait with an inlined first probe (the common, already-complete case).
+__device__ __forceinline__ bool lf_wait_fast(uint32_t bar, uint32_t parity,
+                                             volatile int *abort_flag, int32_t *status, int site) {
+  if (lf_mbar_try(bar, parity)) return true;
+  return lf_wait(bar, parity, abort_flag, status, site);
+}
+
+// Warp-uniform bounded wait: the converged warp polls together (every lane
+// acquires the phase itself), and the verdict is made uniform before the
 // warp-collective tcgen05 instructions that follow.
 __device__ __forceinline__ bool lf_wait_warp(uint32_t bar, uint32_t parity,
                                              volatile int *abort_flag, int32_t *status, int site) {
-  int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = lf_wait(bar, parity, abort_flag, status, site) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  if (ok) {
-    while (!lf_mbar_try(bar, parity)) {
-    }
-  }
-  __syncwarp();
-  return ok != 0;
+  const bool ok = lf_wait_fast(bar, parity, abort_flag, status, site);
+  return __all_sync(0xffffffffu, ok);
 }
 
 __device__ __forceinline__ void lf_tma_load4(uint32_t dst, const CUtensorMap *map, uint32_t bar,
@@ -383,9 +383,26 @@ __device__ __forceinline__ void lf_tmem_ld32x2(uint32_t taddr, float (&x)[32], f
 // p = 2^(s * sl2 - m) into P (TMEM, packed bf16 / f16) and their sum lt.
 // Chunks no lane of the warp attends are skipped (P written as zeros); two
 // attended chunks are fetched with one TMEM wait.
+// Gate before the first write of P (or O) of a tile: the previous tile's
+// P.V must have finished reading P.  `pending` is the pv_done phase still
+// to be observed, or -1.
+struct LfPvGate {
+  uint32_t bar;
+  int pending;
+  volatile int *abort_flag;
+  int32_t *status;
+  __device__ __forceinline__ bool pass() {
+    if (pending < 0) return true;
+    const bool ok = lf_wait_warp(bar, (uint32_t)pending, abort_flag, status, 10);
+    pending = -1;
+    return ok;
+  }
+};
+
 template <int kF16>
 __device__ __forceinline__ void lf_softmax_tile(uint32_t tl, const uint32_t (&w)[4], float sl2,
-                                                float m, float &mx, float &lt, bool write_p) {
+                                                float m, float &mx, float &lt, bool write_p,
+                                                LfPvGate &gate) {
   const float mneg = m == -INFINITY ? 0.f : -m;
 #pragma unroll
   for (int pp = 0; pp < 2; pp++) {
@@ -393,6 +410,7 @@ __device__ __forceinline__ void lf_softmax_tile(uint32_t tl, const uint32_t (&w)
     const bool a0 = __any_sync(0xffffffffu, w[c0] != 0u);
     const bool a1 = __any_sync(0xffffffffu, w[c1] != 0u);
     if (write_p && !(a0 && a1)) {
+      gate.pass();
       uint32_t z[16];
 #pragma unroll
       for (int k = 0; k < 16; k++) z[k] = 0u;
@@ -406,6 +424,7 @@ __device__ __forceinline__ void lf_softmax_tile(uint32_t tl, const uint32_t (&w)
       lf_mask_chunk(y, w[c1]);
       mx = fmaxf(mx, fmaxf(lf_max32(x), lf_max32(y)));
       if (write_p) {
+        gate.pass();
         lf_p_chunk<kF16>(tl, c0, x, sl2, mneg, lt);
         lf_p_chunk<kF16>(tl, c1, y, sl2, mneg, lt);
       }
@@ -415,7 +434,10 @@ __device__ __forceinline__ void lf_softmax_tile(uint32_t tl, const uint32_t (&w)
       lf_tmem_ld32(tl + LF_TM_S + 32 * c, x);
       lf_mask_chunk(x, w[c]);
       mx = fmaxf(mx, lf_max32(x));
-      if (write_p) lf_p_chunk<kF16>(tl, c, x, sl2, mneg, lt);
+      if (write_p) {
+        gate.pass();
+        lf_p_chunk<kF16>(tl, c, x, sl2, mneg, lt);
+      }
     }
   }
 }
@@ -495,8 +517,8 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 2)
   // ---------------------------------------------------- shared state
   const uint32_t bar = sbase + LF_SM_BAR;
   const uint32_t q_full = bar, s_full = bar + 8, p_full = bar + 16, o_full = bar + 24,
-                 end_bar = bar + 32;
-  const uint32_t kv_full0 = bar + 40, kv_empty0 = bar + 40 + 8 * LF_TC_NS;
+                 end_bar = bar + 32, pv_done = bar + 40;
+  const uint32_t kv_full0 = bar + 48, kv_empty0 = bar + 48 + 8 * LF_TC_NS;
   uint32_t *tmem_slot = (uint32_t *)(gbase + LF_SM_BAR + 128);
   volatile int *abort_flag = (volatile int *)(gbase + LF_SM_BAR + 132);
 
@@ -506,6 +528,7 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 2)
     lf_mbar_init(p_full, 4);
     lf_mbar_init(o_full, 1);
     lf_mbar_init(end_bar, 1);
+    lf_mbar_init(pv_done, 1);
     for (int s = 0; s < LF_TC_NS; s++) {
       lf_mbar_init(kv_full0 + 8 * s, 1);
       lf_mbar_init(kv_empty0 + 8 * s, 1);
@@ -565,45 +588,51 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 2)
   } else if (warp == 1) {
     // ================================================== MMA issuer
     if (lane == 0) {
-      const uint32_t id_pv = lf_idesc(kF16, 64, 1);
+      // descriptors: start-address field (16-byte units) advanced per k-step
+      const uint64_t dq = lf_sdesc(sbase + LF_SM_Q, 16, 1024);
+      const uint64_t dk0 = lf_sdesc(sbase + LF_SM_K(0), 16, 1024);
+      const uint64_t dv0 = lf_sdesc(sbase + LF_SM_V(0), 0, 1024);
+      const uint32_t id_pv = lf_idesc(kF16, 64, 1), id_s = lf_idesc(kF16, LF_BK, 0);
       const int ngk = (ng + 15) / 16 * 16;  // global key tile width, multiple of 16
-      auto ncols_of = [&](int it) { return it < nband ? LF_BK : min(LF_BK, ngk - (it - nband) * LF_BK); };
       auto issue_s = [&](int it) {
         const int s = it % LF_TC_NS;
-        const uint32_t id = lf_idesc(kF16, ncols_of(it), 0);
+        const uint64_t dk = dk0 + (uint64_t)(s * (16384 >> 4));
+        const uint32_t id = it < nband ? id_s : lf_idesc(kF16, min(LF_BK, ngk - (it - nband) * LF_BK), 0);
 #pragma unroll
-        for (int k = 0; k < 4; k++) {
-          uint64_t a = lf_sdesc(sbase + LF_SM_Q + 32 * k, 16, 1024);
-          uint64_t bb = lf_sdesc(sbase + LF_SM_K(s) + 32 * k, 16, 1024);
-          lf_mma_ss(tmem + LF_TM_S, a, bb, id, k > 0);
-        }
+        for (int k = 0; k < 4; k++) lf_mma_ss(tmem + LF_TM_S, dq + 2 * k, dk + 2 * k, id, k > 0);
       };
-      bool ok = lf_wait(q_full, 0, abort_flag, D.status, 3) &&
-                lf_wait(kv_full0, 0, abort_flag, D.status, 4);
+      auto issue_pv = [&](int it) {
+        const int s = it % LF_TC_NS;
+        const uint64_t dv = dv0 + (uint64_t)(s * (16384 >> 4));
+        const int ksteps = it < nband ? 8 : min(LF_BK, ngk - (it - nband) * LF_BK) / 16;
+#pragma unroll
+        for (int k = 0; k < 8; k++)
+          if (k < ksteps)
+            lf_mma_ts(tmem + LF_TM_O, tmem + LF_TM_P + 8 * k, dv + 128 * k, id_pv, (it > 0 || k > 0));
+      };
+      bool ok = lf_wait_fast(q_full, 0, abort_flag, D.status, 3) &&
+                lf_wait_fast(kv_full0, 0, abort_flag, D.status, 4);
       if (ok) {
         lf_tc_fence_after();
         issue_s(0);
         lf_tc_commit(s_full);
         for (int it = 0; it < T; it++) {
-          if (!lf_wait(p_full, it & 1, abort_flag, D.status, 5)) break;
+          // P(it) written and S(it) consumed by the softmax warps
+          if (!lf_wait_fast(p_full, it & 1, abort_flag, D.status, 5)) break;
           lf_tc_fence_after();
-          const int s = it % LF_TC_NS;
-          const int ksteps = ncols_of(it) / 16;
-          for (int k = 0; k < ksteps; k++) {
-            uint64_t bb = lf_sdesc(sbase + LF_SM_V(s) + 2048 * k, 0, 1024);
-            lf_mma_ts(tmem + LF_TM_O, tmem + LF_TM_P + 8 * k, bb, id_pv, (it > 0 || k > 0));
-          }
-          lf_tc_commit(kv_empty0 + 8 * s);
           if (it + 1 < T) {
+            // the next scores first: they only need the S columns, now free
             const int s2 = (it + 1) % LF_TC_NS;
-            if (!lf_wait(kv_full0 + 8 * s2, ((it + 1) / LF_TC_NS) & 1, abort_flag, D.status, 6))
+            if (!lf_wait_fast(kv_full0 + 8 * s2, ((it + 1) / LF_TC_NS) & 1, abort_flag, D.status, 6))
               break;
             lf_tc_fence_after();
             issue_s(it + 1);
             lf_tc_commit(s_full);
-          } else {
-            lf_tc_commit(o_full);
           }
+          issue_pv(it);
+          lf_tc_commit(kv_empty0 + 8 * (it % LF_TC_NS));
+          lf_tc_commit(pv_done);  // P columns free again, O up to date
+          if (it + 1 == T) lf_tc_commit(o_full);
         }
       }
       // every MMA this thread issued has completed once end_bar flips
@@ -687,15 +716,16 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 2)
       // ---- probabilities of the tile -> P (TMEM).  Optimistic single pass
       // against the running reference m_ref; redone (rarely) with the tile's
       // own max when some row's max grew by more than 2^8.
+      LfPvGate gate{pv_done, it > 0 ? ((it - 1) & 1) : -1, abort_flag, D.status};
       const bool any_bits = (w[0] | w[1] | w[2] | w[3]) != 0u;
       const bool single = __all_sync(0xffffffffu, m_ref != -INFINITY || !any_bits);
       float mx = -INFINITY, lt = 0.f;
-      if (single) lf_softmax_tile<kF16>(tl, w, sl2, m_ref, mx, lt, true);
+      if (single) lf_softmax_tile<kF16>(tl, w, sl2, m_ref, mx, lt, true, gate);
       const bool grow = any_bits && (!single || mx * sl2 > m_ref + 8.f);
       if (__any_sync(0xffffffffu, grow)) {
         if (!single) {
           float dummy = 0.f;
-          lf_softmax_tile<kF16>(tl, w, sl2, m_ref, mx, dummy, false);  // max only
+          lf_softmax_tile<kF16>(tl, w, sl2, m_ref, mx, dummy, false, gate);  // max only
         }
         const float ms = mx * sl2;
         const bool need = any_bits && ms > m_ref + 8.f;
@@ -703,6 +733,7 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 2)
         const float alpha = need ? lf_ex2(m_ref - m_new) : 1.f;
         l *= alpha;
         if (it > 0 && __any_sync(0xffffffffu, need)) {
+          gate.pass();
 #pragma unroll
           for (int half = 0; half < 2; half++) {
             float ov[32];
@@ -715,9 +746,10 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 2)
         m_ref = m_new;
         lt = 0.f;
         float mx2 = -INFINITY;
-        lf_softmax_tile<kF16>(tl, w, sl2, m_ref, mx2, lt, true);
+        lf_softmax_tile<kF16>(tl, w, sl2, m_ref, mx2, lt, true, gate);
       }
       l += lt;
+      gate.pass();  // (no-op unless every chunk of the tile was skipped)
       lf_tmem_wait_st();
       lf_tc_fence_before();
       __syncwarp();

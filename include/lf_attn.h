@@ -139,6 +139,28 @@ int lf_attn_status(void *workspace, void *stream);
  * Pass NULL, NULL to turn it off. */
 int lf_attn_set_timing_events(void *ev_start, void *ev_stop);
 
+/* Bytes of device scratch built into the library for lf_attn_fwd_noalloc. */
+#define LF_STATIC_WORKSPACE_BYTES (16u << 20)
+
+/* Forward for callers that cannot allocate device memory -- a plugin that
+ * only receives buffers from its host application, or code that must not
+ * call cudaMalloc once it runs.  The pages have no counterpart of this call.
+ * Same computation, arguments and results as lf_attn_fwd, without the
+ * workspace: the scratch is a fixed LF_STATIC_WORKSPACE_BYTES array inside
+ * the library's device image, which every GPU that loads the library holds
+ * until the process exits.  Problems whose lf_attn_workspace_size exceeds it
+ * are rejected with LF_ERR_UNSUPPORTED (use lf_attn_fwd).  The call allocates
+ * nothing.  Its first call on a device looks up the array's device address
+ * (with that device current; `stream` must belong to it); make that first
+ * call before any stream capture.  All calls on a device share the one
+ * array, so calls that may overlap on the GPU (other streams, other host
+ * threads) race and must be serialised by the caller.  The device status
+ * word of this variant is not readable through lf_attn_status. */
+int lf_attn_fwd_noalloc(const lf_attn_params *p, const void *q_s,
+                        const void *k_s, const void *v_s, const void *q_g,
+                        const void *k_g, const void *v_g, const int32_t *mask,
+                        void *o, float *lse, void *stream);
+
 /* Number of kernels this library has launched in this process so far (all
  * threads).  Lets a caller count the kernels inside a timed region. */
 uint64_t lf_attn_launch_count(void);

@@ -29,6 +29,8 @@ static int lf_fail(int code, const char *fmt, ...) {
   return code;
 }
 
+int lf_record_error(int code, const char *msg) { return lf_fail(code, "%s", msg); }
+
 static int lf_cuda(cudaError_t e, const char *what) {
   if (e == cudaSuccess) return LF_OK;
   return lf_fail(LF_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));

@@ -1,0 +1,70 @@
+// lf_static.cu -- lf_attn_fwd_noalloc: the forward for callers that cannot
+// allocate device memory.
+//
+// Some callers only ever receive device buffers from a host application and
+// have no device allocator of their own (a plugin inside an inference engine
+// that owns all device memory), or must not allocate once they are running
+// (cudaMalloc can synchronise the device, and can fail under memory pressure
+// in the middle of serving).  They pass inputs and outputs as usual; the
+// scratch the forward needs lives in a fixed-size array that is part of this
+// library's device image.  Every GPU that loads the library holds
+// LF_STATIC_WORKSPACE_BYTES of device memory for it until the process exits.
+//
+// On the host, the array's name is only a host-side stand-in for the device
+// symbol, never a device address; the device address comes from
+// cudaGetSymbolAddress, once per device, with that device current.
+#include <stdio.h>
+
+#include <mutex>
+
+#include "lf_attn.h"
+
+#define LF_STATIC_MAX_DEVICES 64
+
+static __device__ __align__(256) unsigned char lf_static_ws[LF_STATIC_WORKSPACE_BYTES];
+
+static std::mutex g_static_mu;
+static void *g_static_addr[LF_STATIC_MAX_DEVICES];
+
+// defined in lf_api.cu: record an error for lf_attn_last_error()
+int lf_record_error(int code, const char *msg);
+
+extern "C" int lf_attn_fwd_noalloc(const lf_attn_params *p, const void *q_s, const void *k_s,
+                                   const void *v_s, const void *q_g, const void *k_g,
+                                   const void *v_g, const int32_t *mask, void *o, float *lse,
+                                   void *stream) {
+  const size_t need = lf_attn_workspace_size(p, 0);
+  if (need == 0)  // invalid params: let the regular entry point name the problem
+    return lf_attn_fwd(p, q_s, k_s, v_s, q_g, k_g, v_g, mask, o, lse, nullptr, 0, stream);
+  if (need > (size_t)LF_STATIC_WORKSPACE_BYTES) {
+    char msg[192];
+    snprintf(msg, sizeof(msg),
+             "lf_attn_fwd_noalloc: this problem needs %zu bytes of scratch, the static scratch "
+             "holds %zu; use lf_attn_fwd with a caller-allocated workspace",
+             need, (size_t)LF_STATIC_WORKSPACE_BYTES);
+    return lf_record_error(LF_ERR_UNSUPPORTED, msg);
+  }
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return lf_record_error(LF_ERR_CUDA, "lf_attn_fwd_noalloc: cudaGetDevice failed");
+  if (dev < 0 || dev >= LF_STATIC_MAX_DEVICES)
+    return lf_record_error(LF_ERR_UNSUPPORTED, "lf_attn_fwd_noalloc: device ordinal out of range");
+  void *base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_addr[dev]) {
+      // first call on this device (the current one): look the symbol up
+      void *ptr = nullptr;
+      e = cudaGetSymbolAddress(&ptr, lf_static_ws);
+      if (e != cudaSuccess || !ptr)
+        return lf_record_error(LF_ERR_CUDA, "lf_attn_fwd_noalloc: cudaGetSymbolAddress failed");
+      g_static_addr[dev] = ptr;
+    }
+    base = g_static_addr[dev];
+  }
+  // The regular forward clears the status word at its start and fully
+  // writes every other scratch region before reading it, so the contents a
+  // previous call left behind never matter.
+  return lf_attn_fwd(p, q_s, k_s, v_s, q_g, k_g, v_g, mask, o, lse, base,
+                     (size_t)LF_STATIC_WORKSPACE_BYTES, stream);
+}

@@ -23,7 +23,9 @@ ERROR_NAMES = {1: "LF_ERR_INVALID", 2: "LF_ERR_UNSUPPORTED", 3: "LF_ERR_CUDA",
 # every symbol include/lf_attn.h declares
 EXPORTS = ["lf_attn_version", "lf_attn_workspace_size", "lf_attn_fwd", "lf_attn_bwd",
            "lf_attn_count_pairs", "lf_attn_mask_dump", "lf_attn_status",
-           "lf_attn_set_timing_events", "lf_attn_launch_count", "lf_attn_last_error"]
+           "lf_attn_set_timing_events", "lf_attn_launch_count", "lf_attn_last_error",
+           "lf_attn_fwd_noalloc"]
+LF_STATIC_WORKSPACE_BYTES = 16 << 20
 
 
 class LfError(RuntimeError):
@@ -62,6 +64,8 @@ def load(path: str = LIB_PATH):
         lib.lf_attn_set_timing_events.argtypes = [vp, vp]
         lib.lf_attn_last_error.restype = ctypes.c_char_p
         lib.lf_attn_launch_count.restype = ctypes.c_uint64
+        lib.lf_attn_fwd_noalloc.argtypes = [P] + [vp] * 6 + [vp, vp, vp, vp]
+        lib.lf_attn_fwd_noalloc.restype = i32
         for f in ("fwd", "bwd", "count_pairs", "mask_dump", "status", "set_timing_events"):
             getattr(lib, "lf_attn_" + f).restype = i32
         _lib = lib
@@ -122,6 +126,14 @@ def lf_attn_fwd(p, q_s, k_s, v_s, q_g, k_g, v_g, mask, o, lse, ws, stream=None):
     _check(load().lf_attn_fwd(ctypes.byref(p), _ptr(q_s), _ptr(k_s), _ptr(v_s), _ptr(q_g),
                               _ptr(k_g), _ptr(v_g), _ptr(mask), _ptr(o), _ptr(lse), _ptr(ws),
                               ws.numel(), _stream(stream)))
+
+
+def lf_attn_fwd_noalloc(p, q_s, k_s, v_s, q_g, k_g, v_g, mask, o, lse, stream=None):
+    """Forward without a workspace argument (library-internal static scratch);
+    for callers that cannot allocate device memory."""
+    _check(load().lf_attn_fwd_noalloc(ctypes.byref(p), _ptr(q_s), _ptr(k_s), _ptr(v_s), _ptr(q_g),
+                                      _ptr(k_g), _ptr(v_g), _ptr(mask), _ptr(o), _ptr(lse),
+                                      _stream(stream)))
 
 
 def lf_attn_bwd(p, q_s, k_s, v_s, q_g, k_g, v_g, mask, o, lse, d_o, dq_s, dk_s, dv_s, dq_g, dk_g,

@@ -187,6 +187,43 @@ def cpu_baseline(wl, budget_s=10.0):
             "sample": "%d of %d (b,h) heads of %s, float64, %.1f s" % (done, wl.B * wl.H, wl.name, t_total)}
 
 
+def time_backward(att, d, wl, pairs, world, args, dev, stream):
+    """Time lf_attn_bwd (six gradients) on the forward's outputs; reported
+    beside the forward metric (algorithmic 8 * head_dim FLOP per pair)."""
+    import torch
+    from sparse_sliding_window_b200 import lf_attn as L
+    g = torch.randn_like(d["qs"])
+    if att.ws_b is None:
+        att.ws_b = L.workspace(att.p, True, dev)
+    grads = [torch.empty_like(d["qs"]) for _ in range(6)]
+
+    def bstep():
+        L.lf_attn_bwd(att.p, d["qs"], d["ks"], d["vs"], d["qg"], d["kg"], d["vg"], d["mask"], d["o"],
+                      d["lse"], g, *grads, att.ws_b)
+
+    for _ in range(max(3, args.warmup // 4)):
+        bstep()
+    torch.cuda.synchronize(dev)
+    att.status(bwd=True)
+    k = max(3, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record(stream)
+    for _ in range(k):
+        bstep()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / k
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"ms_per_step": ms, "steps": k, "kernels": "CUDA-core backward (delta, dQ, dK_s/dV_s, dK_g/dV_g)",
+            "tflops_algorithmic": 8.0 * wl.head_dim * pairs * world / (ms * 1e-3) / 1e12,
+            "scores_per_s": pairs * world / (ms * 1e-3)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -197,6 +234,8 @@ def main():
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--min-warm-seconds", type=float, default=1.0)
+    ap.add_argument("--bwd", action="store_true",
+                    help="also time the backward (default for workloads with a backward)")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
@@ -361,6 +400,8 @@ def main():
             "e2e": {"value": pairs * world / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                     "ms_per_step": e2e_ms}}
+    if args.bwd or wl.backward:
+        line["backward"] = time_backward(att, sets[0], wl, pairs, world, args, dev, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:

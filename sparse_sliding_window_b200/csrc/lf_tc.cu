@@ -22,19 +22,27 @@
 //    全局注意力).  Each writes an unnormalised partial (acc, max, sum) that
 //    lf_combine_kernel merges (split-KV).
 //
-// Per CTA (192 threads, two CTAs per SM): warp 0 issues TMA loads (Q once,
-// then K/V tiles into a 2-stage ring), warp 1 owns TMEM and issues the
-// tcgen05.mma instructions, warps 2..5 (one TMEM lane = one query row per
-// thread) run the softmax.  TMEM columns: S = QK^T tile [0,128), the O
-// accumulator [128,192), P (bf16/f16, packed two per column) [192,256).
-// Per tile:   MMA  S_t = Q K_t^T      -> commit s_full
-//             SMX  read S_t, row max, rescale O if the max grew by more than
-//                  2^8, P_t = exp2(S_t*scale*log2e - m), row sum, write P_t
-//                                     -> arrive p_full
-//             MMA  O += P_t V_t (A operand from TMEM) -> commit kv_empty
-//             MMA  S_{t+1} = Q K_{t+1}^T -> commit s_full
-// so the n x w score band never leaves the SM.  The two CTAs of an SM
-// interleave their MMA and softmax phases.
+// Persistent: one CTA of 320 threads per SM walks the work items
+// blockIdx.x, blockIdx.x + gridDim.x, ...  Warp 8 issues TMA loads (Q per
+// item into one of two buffers, K/V tiles into a 5-stage ring that runs
+// ahead into the next item), warp 9 owns all 512 TMEM columns and issues
+// the tcgen05.mma instructions, and two softmax
+// groups of four warps (warps 0-3, 4-7; one TMEM lane = one query row per
+// thread) take the key tiles of an item in turn: group 0 tiles 0, 2, 4, ..., group 1 tiles 1, 3, 5, ...  Each group
+// has its own S tile, O accumulator and P tile in TMEM
+// (S_g = [128g, 128g+128), O_g = [256+64g, +64), P_g = [384+64g, +64)), so
+// one group's softmax overlaps the tensor-core work of the other's.
+// Per tile t of group g:
+//             MMA  S_g = Q K_t^T                       -> commit s_full(g)
+//             SMX  P_g = exp2(S*scale*log2e - m) against the running max m
+//                  (redone with a new m, O_g rescaled, when a row max grew
+//                  by more than 2^8), row sum
+//                                                      -> arrive p_full(g)
+//             MMA  S_g = Q K_{t+2}^T  (next tile of the group) -> s_full(g)
+//             MMA  O_g += P_g V_t (A operand from TMEM) -> kv_empty, pv_done(g)
+// At the end of an item the two groups merge their (max, sum, O) on chip
+// and write O and the log-normaliser, so the n x w score band never leaves
+// the SM.
 //
 // Every wait is bounded: after LF_WAIT_NS without progress the waiting
 // thread records LF_ERR_DEVICE_TIMEOUT in the status word, raises the CTA's
@@ -45,30 +53,33 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <map>
 #include <utility>
 #include <vector>
 
 #include "lf_tc.cuh"
 
-#define LF_TC_THREADS 192
-#define LF_TC_NS 3
+#define LF_TC_THREADS 320
+#define LF_TC_NS 5
 #define LF_TC_MAX_MAPS 28
 #define LF_TC_MAX_SEG 32
 #define LF_WAIT_NS 1500000000ull
 
-// TMEM column map
-#define LF_TM_S 0
-#define LF_TM_O 128
-#define LF_TM_P 192
-#define LF_TM_COLS 256
+// TMEM column map (per softmax group g = 0, 1)
+#define LF_TM_S(g) ((g)*128)
+#define LF_TM_O(g) (256 + (g)*64)
+#define LF_TM_P(g) (384 + (g)*64)
+#define LF_TM_COLS 512
 
-// shared memory map (bytes from the 1024-aligned base)
-#define LF_SM_Q 0
-#define LF_SM_K(s) (16384 + (s)*16384)
-#define LF_SM_V(s) (16384 + LF_TC_NS * 16384 + (s)*16384)
-#define LF_SM_BAR (16384 + 2 * LF_TC_NS * 16384)
-#define LF_SMEM_BYTES (LF_SM_BAR + 256)
+// shared memory map (bytes from the 1024-aligned base): two Q buffers, then
+// LF_TC_NS stages of (K tile, V tile), barriers, the merge exchange
+#define LF_SM_Q(i) ((i)*16384)
+#define LF_SM_K(s) (32768 + (s)*32768)
+#define LF_SM_V(s) (32768 + (s)*32768 + 16384)
+#define LF_SM_BAR (32768 + LF_TC_NS * 32768)
+#define LF_SM_XCH (LF_SM_BAR + 512)
+#define LF_SMEM_BYTES (LF_SM_XCH + 2 * LF_BQ * 8)
 
 struct LfTcSeg {
   int h0, h1, d, rho, cnt, nqb, start, map;
@@ -308,8 +319,72 @@ __device__ __forceinline__ uint32_t lf_range_bits(int lo, int hi, int base) {
 // row max of the attended raw scores in mx; when write_p, also computes
 // p = 2^(s * sl2 - m) into P (TMEM, packed bf16 / f16) and their sum lt.
 // Chunks no lane of the warp attends are skipped (P written as zeros).
+// TMEM load of 32 columns without waiting; the caller waits with
+// lf_tmem_wait_ld_regs, which also pins the registers behind the wait.
+__device__ __forceinline__ void lf_tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void lf_tmem_wait_ld_regs(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
+// packed fp32 pair arithmetic (one instruction for two lanes of data)
+__device__ __forceinline__ uint64_t lf_f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void lf_f2_split(uint64_t v, float &a, float &b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t lf_fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t lf_add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Gate before the first write of P (or O) of a tile: the previous P.V of
+// the same softmax group must have finished reading P.  `pending` is the
+// pv_done phase still to be observed, or -1.
+struct LfPvGate {
+  uint32_t bar;
+  int pending;
+  volatile int *abort_flag;
+  int32_t *status;
+  __device__ __forceinline__ bool pass() {
+    if (pending < 0) return true;
+    const bool ok = lf_wait_warp(bar, (uint32_t)pending, abort_flag, status, 10);
+    pending = -1;
+    return ok;
+  }
+};
+
 template <int kF16>
-__device__ __forceinline__ void lf_p_chunk(uint32_t tl, int cc, float (&x)[32], float sl2,
+__device__ __forceinline__ void lf_p_chunk(uint32_t tP, int cc, float (&x)[32], float sl2,
                                            float mneg, float &lt) {
   uint32_t pw[16];
   float s0 = 0.f, s1 = 0.f;
@@ -322,7 +397,7 @@ __device__ __forceinline__ void lf_p_chunk(uint32_t tl, int cc, float (&x)[32], 
     pw[k / 2] = lf_pack2<kF16>(p0, p1);
   }
   lt += s0 + s1;
-  lf_tmem_st16(tl + LF_TM_P + 16 * cc, pw);
+  lf_tmem_st16(tP + 16 * cc, pw);
 }
 
 __device__ __forceinline__ void lf_mask_chunk(float (&x)[32], uint32_t wc) {
@@ -383,24 +458,9 @@ __device__ __forceinline__ void lf_tmem_ld32x2(uint32_t taddr, float (&x)[32], f
 // p = 2^(s * sl2 - m) into P (TMEM, packed bf16 / f16) and their sum lt.
 // Chunks no lane of the warp attends are skipped (P written as zeros); two
 // attended chunks are fetched with one TMEM wait.
-// Gate before the first write of P (or O) of a tile: the previous tile's
-// P.V must have finished reading P.  `pending` is the pv_done phase still
-// to be observed, or -1.
-struct LfPvGate {
-  uint32_t bar;
-  int pending;
-  volatile int *abort_flag;
-  int32_t *status;
-  __device__ __forceinline__ bool pass() {
-    if (pending < 0) return true;
-    const bool ok = lf_wait_warp(bar, (uint32_t)pending, abort_flag, status, 10);
-    pending = -1;
-    return ok;
-  }
-};
 
 template <int kF16>
-__device__ __forceinline__ void lf_softmax_tile(uint32_t tl, const uint32_t (&w)[4], float sl2,
+__device__ __forceinline__ void lf_softmax_tile(uint32_t tS, uint32_t tP, const uint32_t (&w)[4], float sl2,
                                                 float m, float &mx, float &lt, bool write_p,
                                                 LfPvGate &gate) {
   const float mneg = m == -INFINITY ? 0.f : -m;
@@ -414,130 +474,211 @@ __device__ __forceinline__ void lf_softmax_tile(uint32_t tl, const uint32_t (&w)
       uint32_t z[16];
 #pragma unroll
       for (int k = 0; k < 16; k++) z[k] = 0u;
-      if (!a0) lf_tmem_st16(tl + LF_TM_P + 16 * c0, z);
-      if (!a1) lf_tmem_st16(tl + LF_TM_P + 16 * c1, z);
+      if (!a0) lf_tmem_st16(tP + 16 * c0, z);
+      if (!a1) lf_tmem_st16(tP + 16 * c1, z);
     }
     if (a0 && a1) {
       float x[32], y[32];
-      lf_tmem_ld32x2(tl + LF_TM_S + 32 * c0, x, y);
+      lf_tmem_ld32x2(tS + 32 * c0, x, y);
       lf_mask_chunk(x, w[c0]);
       lf_mask_chunk(y, w[c1]);
       mx = fmaxf(mx, fmaxf(lf_max32(x), lf_max32(y)));
       if (write_p) {
         gate.pass();
-        lf_p_chunk<kF16>(tl, c0, x, sl2, mneg, lt);
-        lf_p_chunk<kF16>(tl, c1, y, sl2, mneg, lt);
+        lf_p_chunk<kF16>(tP, c0, x, sl2, mneg, lt);
+        lf_p_chunk<kF16>(tP, c1, y, sl2, mneg, lt);
       }
     } else if (a0 || a1) {
       const int c = a0 ? c0 : c1;
       float x[32];
-      lf_tmem_ld32(tl + LF_TM_S + 32 * c, x);
+      lf_tmem_ld32(tS + 32 * c, x);
       lf_mask_chunk(x, w[c]);
       mx = fmaxf(mx, lf_max32(x));
       if (write_p) {
         gate.pass();
-        lf_p_chunk<kF16>(tl, c, x, sl2, mneg, lt);
+        lf_p_chunk<kF16>(tP, c, x, sl2, mneg, lt);
       }
     }
   }
 }
 
+// P for one S tile of this thread's TMEM lane against the reference m:
+// p = 2^(s*sl2 - m) for the attended columns (bit set in w), 0 elsewhere,
+// packed into P, summed into lt; with want_max the attended max of the raw
+// scores goes to mx instead and nothing is written.  TMEM loads run one
+// 32-column chunk ahead of the arithmetic; the arithmetic of chunks no lane
+// of the warp attends is skipped (P written as zeros).
+template <int kF16>
+__device__ __forceinline__ void lf_tile_pass(uint32_t tS, uint32_t tP, const uint32_t (&w)[4],
+                                             float sl2, float m, float &lt, float &mx,
+                                             bool want_max, LfPvGate &gate) {
+  bool anyc[4];
+#pragma unroll
+  for (int cc = 0; cc < 4; cc++) anyc[cc] = __any_sync(0xffffffffu, w[cc] != 0u);
+  const float mneg = -m;
+  uint32_t buf[2][32];  // chunk cc lives in buf[cc & 1]; chunk cc+1 loads while cc computes
+  float s0 = 0.f, s1 = 0.f, m0 = -INFINITY, m1 = -INFINITY;
+  lf_tmem_ld32_nowait(tS, buf[0]);
+#pragma unroll
+  for (int cc = 0; cc < 4; cc++) {
+    uint32_t(&x)[32] = buf[cc & 1];
+    lf_tmem_wait_ld_regs(x);
+    if (cc + 1 < 4) lf_tmem_ld32_nowait(tS + 32 * (cc + 1), buf[(cc + 1) & 1]);
+    if (!anyc[cc]) {
+      if (!want_max) {
+        gate.pass();
+        uint32_t z[16];
+#pragma unroll
+        for (int k = 0; k < 16; k++) z[k] = 0u;
+        lf_tmem_st16(tP + 16 * cc, z);
+      }
+      continue;
+    }
+    const uint32_t wc = w[cc];
+    if (!__all_sync(0xffffffffu, wc == 0xffffffffu)) {
+#pragma unroll
+      for (int k = 0; k < 32; k++) x[k] = ((wc >> k) & 1u) ? x[k] : 0xff800000u;  // -inf
+    }
+    if (want_max) {
+#pragma unroll
+      for (int k = 0; k < 32; k += 2) {
+        m0 = fmaxf(m0, __uint_as_float(x[k]));
+        m1 = fmaxf(m1, __uint_as_float(x[k + 1]));
+      }
+    } else {
+      uint32_t pw[16];
+#pragma unroll
+      for (int k = 0; k < 32; k += 2) {
+        const float p0 = lf_ex2(fmaf(__uint_as_float(x[k]), sl2, mneg));
+        const float p1 = lf_ex2(fmaf(__uint_as_float(x[k + 1]), sl2, mneg));
+        s0 += p0;
+        s1 += p1;
+        pw[k / 2] = lf_pack2<kF16>(p0, p1);
+      }
+      gate.pass();
+      lf_tmem_st16(tP + 16 * cc, pw);
+    }
+  }
+  if (want_max) mx = fmaxf(m0, m1);
+  else lt = s0 + s1;
+}
+
+// A decoded work item (every role decodes the same sequence).
+struct LfItem {
+  int gitem, b, h, d, rho, cnt, qrow0, mq, mk, mv, nband, nglob, T, kt0, ng;
+};
+
+__device__ __forceinline__ bool lf_decode(const LfTcParams &P, int idx, LfItem &it) {
+  const LfDev &D = P.dev;
+  const int n = D.n;
+  it.d = 1;
+  it.rho = 0;
+  it.cnt = n;
+  it.kt0 = 0;
+  it.nglob = 0;
+  if (idx < P.n_gitems) {
+    it.gitem = 1;
+    const int c = idx % D.nch;
+    idx /= D.nch;
+    const int qt = idx % P.ngq;
+    idx /= P.ngq;
+    it.h = idx % D.H;
+    it.b = idx / D.H;
+    it.ng = D.binfo[(size_t)it.b * LF_BI_WORDS + LF_BI_NG];
+    it.qrow0 = qt * LF_BQ;
+    it.kt0 = c * D.chunk_tiles;
+    const int ktiles = (n + LF_BK - 1) / LF_BK;
+    it.nband = min(D.chunk_tiles, ktiles - it.kt0);
+    it.mq = P.map_qgc;
+    it.mk = P.map_kg;
+    it.mv = P.map_vg;
+    it.T = it.nband;
+    return it.qrow0 < it.ng && it.nband > 0;  // false: nothing to do
+  }
+  it.gitem = 0;
+  idx -= P.n_gitems;
+  it.b = idx / P.per_batch;
+  int rem = idx - it.b * P.per_batch;
+  int s = 0;
+  while (s + 1 < P.nseg && rem >= P.seg[s + 1].start) s++;
+  const LfTcSeg &sg = P.seg[s];
+  rem -= sg.start;
+  it.h = sg.h0 + rem / sg.nqb;
+  it.qrow0 = (rem % sg.nqb) * LF_BQ;
+  it.d = sg.d;
+  it.rho = sg.rho;
+  it.cnt = sg.cnt;
+  it.mq = sg.map;
+  it.mk = sg.map + 1;
+  it.mv = sg.map + 2;
+  it.nband = lf_band_tiles(D.r, D.causal);
+  const int32_t *bi = D.binfo + (size_t)it.b * LF_BI_WORDS;
+  it.ng = bi[LF_BI_NG];
+  bool need = it.ng > 0;
+  if (need && it.d == 1 && !D.causal) {
+    // every global key inside every row's window: the band covers them
+    const int tlast = min(it.qrow0 + LF_BQ - 1, it.cnt - 1);
+    if (bi[LF_BI_GMIN] >= tlast - D.r && bi[LF_BI_GMAX] <= it.qrow0 + D.r) need = false;
+  }
+  it.nglob = need ? (it.ng + LF_BK - 1) / LF_BK : 0;
+  it.T = it.nband + it.nglob;
+  return true;
+}
+
 // ------------------------------------------------------------ the kernel
 
 template <int kF16>
-__global__ void __launch_bounds__(LF_TC_THREADS, 2)
+__global__ void __launch_bounds__(LF_TC_THREADS, 1)
     lf_tc_fwd_kernel(const __grid_constant__ LfTcParams P) {
   extern __shared__ __align__(1024) uint8_t lf_smem_raw[];
   // the dynamic shared window starts 1024-byte aligned (128-byte swizzled
-  // TMA tiles need it); checked rather than padded, to fit two CTAs per SM
+  // TMA tiles need it); checked rather than padded
   const uint32_t sbase = lf_smem(lf_smem_raw);
   uint8_t *gbase = lf_smem_raw;
   if (sbase & 1023u) {
     if (threadIdx.x == 0) lf_set_status(P.dev.status, LF_ERR_UNSUPPORTED, 9000);
     return;
   }
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const LfDev &D = P.dev;
   const int n = D.n;
+  const int nitems = P.n_gitems + D.B * P.per_batch;
 
-  // ---------------------------------------------------- decode work item
-  bool gitem = (int)blockIdx.x < P.n_gitems;
-  int b, h, d = 1, rho = 0, cnt = n, t0 = 0, mq, mk, mv, nband = 0, nglob = 0, kt0 = 0;
-  int ng, qrow0;
-  if (gitem) {
-    int idx = blockIdx.x;
-    const int c = idx % D.nch;
-    idx /= D.nch;
-    const int qt = idx % P.ngq;
-    idx /= P.ngq;
-    h = idx % D.H;
-    b = idx / D.H;
-    ng = D.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
-    if (qt * LF_BQ >= ng) return;  // uniform: no global row in this tile
-    qrow0 = qt * LF_BQ;
-    kt0 = c * D.chunk_tiles;
-    const int ktiles = (n + LF_BK - 1) / LF_BK;
-    nband = min(D.chunk_tiles, ktiles - kt0);
-    if (nband <= 0) return;
-    mq = P.map_qgc;
-    mk = P.map_kg;
-    mv = P.map_vg;
-  } else {
-    int idx = blockIdx.x - P.n_gitems;
-    b = idx / P.per_batch;
-    int rem = idx - b * P.per_batch;
-    int s = 0;
-    while (s + 1 < P.nseg && rem >= P.seg[s + 1].start) s++;
-    const LfTcSeg &sg = P.seg[s];
-    rem -= sg.start;
-    h = sg.h0 + rem / sg.nqb;
-    t0 = (rem % sg.nqb) * LF_BQ;
-    d = sg.d;
-    rho = sg.rho;
-    cnt = sg.cnt;
-    mq = mk = mv = sg.map;  // q, k, v maps at map, map+1, map+2
-    mk += 1;
-    mv += 2;
-    qrow0 = t0;
-    nband = lf_band_tiles(D.r, D.causal);
-    const int32_t *bi = D.binfo + (size_t)b * LF_BI_WORDS;
-    ng = bi[LF_BI_NG];
-    bool need = ng > 0;
-    if (need && d == 1 && !D.causal) {
-      // every global key inside every row's window: the band covers them
-      const int tlast = min(t0 + LF_BQ - 1, cnt - 1);
-      if (bi[LF_BI_GMIN] >= tlast - D.r && bi[LF_BI_GMAX] <= t0 + D.r) need = false;
-    }
-    nglob = need ? (ng + LF_BK - 1) / LF_BK : 0;
-  }
-  const int T = nband + nglob;
-  const int tk0 = t0 - D.r;  // first key row of band tile 0 (sub-sequence coords)
-
-  // ---------------------------------------------------- shared state
+  // barriers (8 bytes each)
   const uint32_t bar = sbase + LF_SM_BAR;
-  const uint32_t q_full = bar, s_full = bar + 8, p_full = bar + 16, o_full = bar + 24,
-                 end_bar = bar + 32, pv_done = bar + 40;
-  const uint32_t kv_full0 = bar + 48, kv_empty0 = bar + 48 + 8 * LF_TC_NS;
-  uint32_t *tmem_slot = (uint32_t *)(gbase + LF_SM_BAR + 128);
-  volatile int *abort_flag = (volatile int *)(gbase + LF_SM_BAR + 132);
+  const uint32_t q_full0 = bar, q_empty0 = bar + 16, kv_full0 = bar + 32,
+                 kv_empty0 = bar + 32 + 8 * LF_TC_NS;
+  const uint32_t gb0 = bar + 32 + 16 * LF_TC_NS;  // per-group barriers, 5 x 2
+  auto s_full = [&](int g) { return gb0 + 8 * g; };
+  auto p_full = [&](int g) { return gb0 + 16 + 8 * g; };
+  auto pv_done = [&](int g) { return gb0 + 32 + 8 * g; };
+  auto o_full = [&](int g) { return gb0 + 48 + 8 * g; };
+  const uint32_t mrg0 = gb0 + 64, mrg1 = gb0 + 72, end_bar = gb0 + 80;
+  uint32_t *tmem_slot = (uint32_t *)(gbase + LF_SM_BAR + 448);
+  volatile int *abort_flag = (volatile int *)(gbase + LF_SM_BAR + 452);
+  float2 *xch = (float2 *)(gbase + LF_SM_XCH);  // [2][128] (max, sum) per group and row
 
   if (threadIdx.x == 0) {
-    lf_mbar_init(q_full, 1);
-    lf_mbar_init(s_full, 1);
-    lf_mbar_init(p_full, 4);
-    lf_mbar_init(o_full, 1);
-    lf_mbar_init(end_bar, 1);
-    lf_mbar_init(pv_done, 1);
+    for (int i = 0; i < 2; i++) {
+      lf_mbar_init(q_full0 + 8 * i, 1);
+      lf_mbar_init(q_empty0 + 8 * i, 1);
+      lf_mbar_init(s_full(i), 1);
+      lf_mbar_init(p_full(i), 4);
+      lf_mbar_init(pv_done(i), 1);
+      lf_mbar_init(o_full(i), 1);
+    }
     for (int s = 0; s < LF_TC_NS; s++) {
       lf_mbar_init(kv_full0 + 8 * s, 1);
       lf_mbar_init(kv_empty0 + 8 * s, 1);
     }
+    lf_mbar_init(mrg0, 8);
+    lf_mbar_init(mrg1, 8);
+    lf_mbar_init(end_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 1) {
+  if (warp == 9) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      lf_smem(tmem_slot)),
                  "r"(LF_TM_COLS)
@@ -549,266 +690,359 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 2)
   lf_tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == 8) {
     // ================================================== TMA producer
     if (lane == 0) {
-      lf_mbar_expect_tx(q_full, 16384);
-      lf_tma_load4(sbase + LF_SM_Q, &P.maps[mq], q_full, 0, qrow0, h, b);
-      int issued = 0;
-      for (int it = 0; it < T; it++) {
-        const int s = it % LF_TC_NS;
-        if (it >= LF_TC_NS &&
-            !lf_wait(kv_empty0 + 8 * s, ((it / LF_TC_NS) & 1) ^ 1, abort_flag, D.status, 1))
+      int gt = 0, k = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < nitems && ok; idx += gridDim.x) {
+        LfItem it;
+        if (!lf_decode(P, idx, it)) continue;
+        const int qb = k & 1;
+        if (k >= 2 && !lf_wait_fast(q_empty0 + 8 * qb, ((k >> 1) & 1) ^ 1, abort_flag, D.status, 1)) {
+          ok = false;
           break;
-        int row;
-        const CUtensorMap *km, *vm;
-        uint32_t bytes;
-        if (it < nband) {
-          row = gitem ? (kt0 + it) * LF_BK : tk0 + it * LF_BK;
-          km = &P.maps[mk];
-          vm = &P.maps[mv];
-          bytes = 2 * 16384;
-        } else {
-          row = (it - nband) * LF_BK;
-          km = &P.maps[P.map_ksc];
-          vm = &P.maps[P.map_vsc];
-          bytes = 2 * P.gbox * 128;
         }
-        lf_mbar_expect_tx(kv_full0 + 8 * s, bytes);
-        lf_tma_load4(sbase + LF_SM_K(s), km, kv_full0 + 8 * s, 0, row, h, b);
-        lf_tma_load4(sbase + LF_SM_V(s), vm, kv_full0 + 8 * s, 0, row, h, b);
-        issued = it + 1;
+        lf_mbar_expect_tx(q_full0 + 8 * qb, 16384);
+        lf_tma_load4(sbase + LF_SM_Q(qb), &P.maps[it.mq], q_full0 + 8 * qb, 0, it.qrow0, it.h, it.b);
+        const int tk0 = it.qrow0 - D.r;
+        for (int t = 0; t < it.T; t++, gt++) {
+          const int s = gt % LF_TC_NS;
+          if (gt >= LF_TC_NS &&
+              !lf_wait_fast(kv_empty0 + 8 * s, ((gt / LF_TC_NS) & 1) ^ 1, abort_flag, D.status, 2)) {
+            ok = false;
+            break;
+          }
+          int row;
+          const CUtensorMap *km, *vm;
+          uint32_t bytes;
+          if (t < it.nband) {
+            row = it.gitem ? (it.kt0 + t) * LF_BK : tk0 + t * LF_BK;
+            km = &P.maps[it.mk];
+            vm = &P.maps[it.mv];
+            bytes = 2 * 16384;
+          } else {
+            row = (t - it.nband) * LF_BK;
+            km = &P.maps[P.map_ksc];
+            vm = &P.maps[P.map_vsc];
+            bytes = 2 * P.gbox * 128;
+          }
+          lf_mbar_expect_tx(kv_full0 + 8 * s, bytes);
+          lf_tma_load4(sbase + LF_SM_K(s), km, kv_full0 + 8 * s, 0, row, it.h, it.b);
+          lf_tma_load4(sbase + LF_SM_V(s), vm, kv_full0 + 8 * s, 0, row, it.h, it.b);
+        }
+        k++;
       }
       if (*abort_flag) {
         // let the copies already issued land before the CTA exits
-        for (int it = max(0, issued - LF_TC_NS); it < issued; it++)
-          lf_wait(kv_full0 + 8 * (it % LF_TC_NS), (it / LF_TC_NS) & 1, abort_flag, D.status, 2);
+        for (int i = max(0, gt - LF_TC_NS); i < gt; i++)
+          lf_wait(kv_full0 + 8 * (i % LF_TC_NS), (i / LF_TC_NS) & 1, abort_flag, D.status, 11);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 9) {
     // ================================================== MMA issuer
     if (lane == 0) {
-      // descriptors: start-address field (16-byte units) advanced per k-step
-      const uint64_t dq = lf_sdesc(sbase + LF_SM_Q, 16, 1024);
+      const uint64_t dq0 = lf_sdesc(sbase + LF_SM_Q(0), 16, 1024);
       const uint64_t dk0 = lf_sdesc(sbase + LF_SM_K(0), 16, 1024);
       const uint64_t dv0 = lf_sdesc(sbase + LF_SM_V(0), 0, 1024);
       const uint32_t id_pv = lf_idesc(kF16, 64, 1), id_s = lf_idesc(kF16, LF_BK, 0);
-      const int ngk = (ng + 15) / 16 * 16;  // global key tile width, multiple of 16
-      auto issue_s = [&](int it) {
-        const int s = it % LF_TC_NS;
-        const uint64_t dk = dk0 + (uint64_t)(s * (16384 >> 4));
-        const uint32_t id = it < nband ? id_s : lf_idesc(kF16, min(LF_BK, ngk - (it - nband) * LF_BK), 0);
+      int gt = 0, k = 0, pc[2] = {0, 0};
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < nitems && ok; idx += gridDim.x) {
+        LfItem it;
+        if (!lf_decode(P, idx, it)) continue;
+        const int qb = k & 1;
+        const int ngk = (it.ng + 15) / 16 * 16;  // global key tile width, multiple of 16
+        auto ncols = [&](int t) { return t < it.nband ? LF_BK : min(LF_BK, ngk - (t - it.nband) * LF_BK); };
+        auto issue_s = [&](int t) {
+          const int s = (gt + t) % LF_TC_NS, g = t & 1;
+          const uint64_t dq = dq0 + (uint64_t)(qb * (16384 >> 4));
+          const uint64_t dk = dk0 + (uint64_t)(s * (32768 >> 4));
+          const uint32_t id = t < it.nband ? id_s : lf_idesc(kF16, ncols(t), 0);
 #pragma unroll
-        for (int k = 0; k < 4; k++) lf_mma_ss(tmem + LF_TM_S, dq + 2 * k, dk + 2 * k, id, k > 0);
-      };
-      auto issue_pv = [&](int it) {
-        const int s = it % LF_TC_NS;
-        const uint64_t dv = dv0 + (uint64_t)(s * (16384 >> 4));
-        const int ksteps = it < nband ? 8 : min(LF_BK, ngk - (it - nband) * LF_BK) / 16;
-#pragma unroll
-        for (int k = 0; k < 8; k++)
-          if (k < ksteps)
-            lf_mma_ts(tmem + LF_TM_O, tmem + LF_TM_P + 8 * k, dv + 128 * k, id_pv, (it > 0 || k > 0));
-      };
-      bool ok = lf_wait_fast(q_full, 0, abort_flag, D.status, 3) &&
-                lf_wait_fast(kv_full0, 0, abort_flag, D.status, 4);
-      if (ok) {
-        lf_tc_fence_after();
-        issue_s(0);
-        lf_tc_commit(s_full);
-        for (int it = 0; it < T; it++) {
-          // P(it) written and S(it) consumed by the softmax warps
-          if (!lf_wait_fast(p_full, it & 1, abort_flag, D.status, 5)) break;
-          lf_tc_fence_after();
-          if (it + 1 < T) {
-            // the next scores first: they only need the S columns, now free
-            const int s2 = (it + 1) % LF_TC_NS;
-            if (!lf_wait_fast(kv_full0 + 8 * s2, ((it + 1) / LF_TC_NS) & 1, abort_flag, D.status, 6))
-              break;
-            lf_tc_fence_after();
-            issue_s(it + 1);
-            lf_tc_commit(s_full);
-          }
-          issue_pv(it);
-          lf_tc_commit(kv_empty0 + 8 * (it % LF_TC_NS));
-          lf_tc_commit(pv_done);  // P columns free again, O up to date
-          if (it + 1 == T) lf_tc_commit(o_full);
+          for (int kk = 0; kk < 4; kk++)
+            lf_mma_ss(tmem + LF_TM_S(g), dq + 2 * kk, dk + 2 * kk, id, kk > 0);
+        };
+        if (!lf_wait_fast(q_full0 + 8 * qb, (k >> 1) & 1, abort_flag, D.status, 3)) {
+          ok = false;
+          break;
         }
+        for (int t = 0; t < 2 && t < it.T; t++) {
+          const int s = (gt + t) % LF_TC_NS;
+          if (!lf_wait_fast(kv_full0 + 8 * s, ((gt + t) / LF_TC_NS) & 1, abort_flag, D.status, 4)) {
+            ok = false;
+            break;
+          }
+          lf_tc_fence_after();
+          issue_s(t);
+          lf_tc_commit(s_full(t & 1));
+        }
+        for (int t = 0; t < it.T && ok; t++) {
+          const int g = t & 1;
+          // P(t) written and S(t) consumed by softmax group g
+          if (!lf_wait_fast(p_full(g), pc[g] & 1, abort_flag, D.status, 5)) {
+            ok = false;
+            break;
+          }
+          pc[g]++;
+          lf_tc_fence_after();
+          if (t + 2 < it.T) {
+            // the group's next scores first: they only need its S columns, now free
+            const int s2 = (gt + t + 2) % LF_TC_NS;
+            if (!lf_wait_fast(kv_full0 + 8 * s2, ((gt + t + 2) / LF_TC_NS) & 1, abort_flag,
+                              D.status, 6)) {
+              ok = false;
+              break;
+            }
+            lf_tc_fence_after();
+            issue_s(t + 2);
+            lf_tc_commit(s_full(g));
+          }
+          const int s = (gt + t) % LF_TC_NS;
+          const uint64_t dv = dv0 + (uint64_t)(s * (32768 >> 4));
+          const int ksteps = ncols(t) / 16;
+#pragma unroll
+          for (int kk = 0; kk < 8; kk++)
+            if (kk < ksteps)
+              lf_mma_ts(tmem + LF_TM_O(g), tmem + LF_TM_P(g) + 8 * kk, dv + 128 * kk, id_pv,
+                        (t >= 2 || kk > 0));
+          lf_tc_commit(kv_empty0 + 8 * s);
+          lf_tc_commit(pv_done(g));  // P columns of group g free again
+          if (t + 2 >= it.T) lf_tc_commit(o_full(g));  // group g's last tile of the item
+        }
+        if (ok) lf_tc_commit(q_empty0 + 8 * qb);  // every S of this item issued
+        k++;
+        gt += it.T;
       }
       // every MMA this thread issued has completed once end_bar flips
       lf_tc_commit(end_bar);
       lf_wait(end_bar, 0, abort_flag, D.status, 7);
     }
-  } else {
-    // ================================================== softmax warps
+  } else if (warp < 8) {
+    // ================================================== softmax groups
+    // warps 0..3 = group 0, warps 4..7 = group 1; group g takes tiles t = g, g+2, ...
+    const int g = warp >> 2;
     const int quarter = warp & 3;
     const int q = quarter * 32 + lane;  // query row of the tile == TMEM lane
-    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int32_t *mrow = D.mask + (size_t)b * n;
-    int code = 0, pos = 0;
-    bool active;
-    if (gitem) {
-      active = qrow0 + q < ng;
-    } else {
-      const int t = t0 + q;
-      if (t < cnt) {
-        pos = rho + t * d;
-        code = mrow[pos];
-      }
-      active = (code == 1);
-    }
-    const int32_t *gl = D.gidx + (size_t)b * D.G;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + LF_TM_S(g), tP = tmem + lane_off + LF_TM_P(g);
+    const uint32_t tO = tmem + lane_off + LF_TM_O(g);
     const float sl2 = D.scale_log2;
-    const bool padded = D.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NVALID] < n;
-    // Global keys already in this row's window: positions [pos - r d, pos + r d]
-    // (causal: up to pos) of the row's residue.  gidx is sorted, so they form
-    // the index range [e_lo, e_hi) = [rank(pos - r d), rank(pos + r d + 1)),
-    // filtered by residue.
-    int e_lo = 0, e_hi = 0;
-    if (!gitem && nglob > 0 && active) {
-      const int32_t *gr = D.grank + (size_t)b * (n + 1);
-      const int lo_pos = max(pos - D.r * d, 0);
-      const int hi_pos = min((D.causal ? pos : pos + D.r * d) + 1, n);
-      e_lo = gr[lo_pos];
-      e_hi = gr[hi_pos];
-    }
-    float m_ref = -INFINITY, l = 0.f;
+    int sc = 0, oc = 0, k = 0;
     bool alive = true;
-    for (int it = 0; it < T && alive; it++) {
-      if (!lf_wait_warp(s_full, it & 1, abort_flag, D.status, 8)) {
+    for (int idx = blockIdx.x; idx < nitems && alive; idx += gridDim.x) {
+      LfItem it;
+      if (!lf_decode(P, idx, it)) continue;
+      const int32_t *mrow = D.mask + (size_t)it.b * n;
+      const int32_t *gl = D.gidx + (size_t)it.b * D.G;
+      int code = 0, pos = 0;
+      bool active;
+      if (it.gitem) {
+        active = it.qrow0 + q < it.ng;
+      } else {
+        const int t = it.qrow0 + q;
+        if (t < it.cnt) {
+          pos = it.rho + t * it.d;
+          code = mrow[pos];
+        }
+        active = (code == 1);
+      }
+      const bool padded = D.binfo[(size_t)it.b * LF_BI_WORDS + LF_BI_NVALID] < n;
+      // global keys already in the row's window: index range [e_lo, e_hi) of
+      // the sorted global list, from the rank array (filtered by residue)
+      int e_lo = 0, e_hi = 0;
+      if (!it.gitem && it.nglob > 0 && active) {
+        const int32_t *gr = D.grank + (size_t)it.b * (n + 1);
+        e_lo = gr[max(pos - D.r * it.d, 0)];
+        e_hi = gr[min((D.causal ? pos : pos + D.r * it.d) + 1, n)];
+      }
+      const int tk0 = it.qrow0 - D.r;
+      float m_ref = 0.f, l = 0.f;
+      for (int t = g; t < it.T; t += 2) {
+        if (!lf_wait_warp(s_full(g), sc & 1, abort_flag, D.status, 8)) {
+          alive = false;
+          break;
+        }
+        lf_tc_fence_after();
+        // ---- attend mask of row q over the tile's 128 columns (4 words)
+        uint32_t w[4];
+        if (t < it.nband) {
+          const int kb = it.gitem ? (it.kt0 + t) * LF_BK : tk0 + t * LF_BK;
+          int lo = 0, hi = LF_BK - 1;
+          if (!it.gitem) lf_band_cols(q, t, D.r, D.causal, lo, hi);
+          lo = max(lo, -kb);  // keys exist on [0, cnt)
+          hi = min(hi, it.cnt - 1 - kb);
+          if (!active) hi = -1;
+#pragma unroll
+          for (int cc = 0; cc < 4; cc++) w[cc] = lf_range_bits(lo, hi, 32 * cc);
+          if (padded) {
+#pragma unroll
+            for (int cc = 0; cc < 4; cc++) {
+              const int tk = kb + 32 * cc + lane;
+              const bool okk = tk >= 0 && tk < it.cnt && mrow[it.rho + tk * it.d] != 0;
+              w[cc] &= __ballot_sync(0xffffffffu, okk);
+            }
+          }
+        } else {
+          const int gbs = (t - it.nband) * LF_BK;
+          const int hi = active ? min(LF_BK - 1, it.ng - 1 - gbs) : -1;
+#pragma unroll
+          for (int cc = 0; cc < 4; cc++) {
+            uint32_t inwin = lf_range_bits(e_lo - gbs, e_hi - 1 - gbs, 32 * cc);
+            if (it.d > 1) {
+              const int e = gbs + 32 * cc + lane;
+              const bool res = e < it.ng && (gl[e] - it.rho) % it.d == 0;
+              inwin &= __ballot_sync(0xffffffffu, res);
+            }
+            w[cc] = lf_range_bits(0, hi, 32 * cc) & ~inwin;
+          }
+        }
+        // ---- probabilities of the tile -> P_g (TMEM) against the running
+        // reference m_ref (0 until a tile says otherwise).  The tile's row sum
+        // shows when the reference is off: a sum above 2^15 means some p may
+        // exceed the P format (f16) -- the row max grew; a sum below 2^-30
+        // on a row whose running sum is also that small means underflow.
+        // Either way the warp redoes the tile with the tile's own max (O_g
+        // rescaled).  S_g stays valid until this group's P is handed over.
+        LfPvGate gate{pv_done(g), sc > 0 ? ((sc - 1) & 1) : -1, abort_flag, D.status};
+        const bool any_bits = (w[0] | w[1] | w[2] | w[3]) != 0u;
+        float lt = 0.f, mx = -INFINITY;
+        lf_tile_pass<kF16>(tS, tP, w, sl2, m_ref, lt, mx, false, gate);
+        const bool off = any_bits && (lt > 32768.f || (lt < 9.3e-10f && l < 9.3e-10f));
+        if (__any_sync(0xffffffffu, off)) {
+          lf_tile_pass<kF16>(tS, tP, w, sl2, m_ref, lt, mx, true, gate);  // max only
+          const float ms = mx * sl2;
+          const bool need = off && ms > -INFINITY;
+          const float m_new = need ? ms : m_ref;
+          const float alpha = need ? lf_ex2(m_ref - m_new) : 1.f;
+          l *= alpha;
+          if (t >= 2 && __any_sync(0xffffffffu, need)) {
+            gate.pass();
+#pragma unroll
+            for (int half = 0; half < 2; half++) {
+              float ov[32];
+              lf_tmem_ld32(tO + 32 * half, ov);
+#pragma unroll
+              for (int kk = 0; kk < 32; kk++) ov[kk] *= alpha;
+              lf_tmem_st32(tO + 32 * half, ov);
+            }
+          }
+          m_ref = m_new;
+          lf_tile_pass<kF16>(tS, tP, w, sl2, m_ref, lt, mx, false, gate);
+        }
+        l += lt;
+        gate.pass();  // (no-op unless every chunk of the tile was skipped)
+        sc++;
+        lf_tmem_wait_st();
+        lf_tc_fence_before();
+        __syncwarp();
+        if (lane == 0) lf_mbar_arrive(p_full(g));
+      }
+      if (!alive) break;
+      // ---- merge the two groups' partial results of this item, write O
+      const bool has_g = it.T > g, has_o = it.T > 1 - g;
+      if (has_g) {
+        if (!lf_wait_warp(o_full(g), oc & 1, abort_flag, D.status, 9)) {
+          alive = false;
+          break;
+        }
+        oc++;
+      }
+      xch[g * LF_BQ + q] = make_float2(m_ref, l);
+      __syncwarp();
+      if (lane == 0) lf_mbar_arrive(mrg0);
+      if (!lf_wait_warp(mrg0, k & 1, abort_flag, D.status, 12)) {
         alive = false;
         break;
       }
       lf_tc_fence_after();
-      // ---- attend mask of row q over the tile's 128 columns (4 words)
-      uint32_t w[4];
-      if (it < nband) {
-        const int kb = gitem ? (kt0 + it) * LF_BK : tk0 + it * LF_BK;
-        int lo = 0, hi = LF_BK - 1;
-        if (!gitem) lf_band_cols(q, it, D.r, D.causal, lo, hi);
-        lo = max(lo, -kb);            // keys exist on [0, cnt)
-        hi = min(hi, cnt - 1 - kb);
-        if (!active) hi = -1;
+      const float2 me = xch[g * LF_BQ + q], ot = xch[(1 - g) * LF_BQ + q];
+      const float mA = g == 0 ? me.x : ot.x, lA = g == 0 ? me.y : ot.y;
+      const float mB = g == 0 ? ot.x : me.x, lB = g == 0 ? ot.y : me.y;
+      const bool hasA = it.T > 0, hasB = it.T > 1;
+      // reference of the merged row: the larger of the groups that summed anything
+      const float M = (lA > 0.f && lB > 0.f) ? fmaxf(mA, mB) : (lA > 0.f ? mA : (lB > 0.f ? mB : 0.f));
+      const float fA = (!hasA || lA <= 0.f) ? 0.f : lf_ex2(mA - M);
+      const float fB = (!hasB || lB <= 0.f) ? 0.f : lf_ex2(mB - M);
+      const float L = lA * fA + lB * fB;
+      // this group writes head-dim columns [32g, 32g + 32), 16 at a time
+      const size_t bh = (size_t)it.b * D.H + it.h;
+      const bool store_row = it.gitem ? active : (it.qrow0 + q < it.cnt && code != 2);
+      const float inv = (!it.gitem && code == 1 && L > 0.f) ? 1.f / L : (it.gitem ? 1.f : 0.f);
+      const float ca = fA * inv, cb = fB * inv;
+      size_t pi = 0, orow = 0;
+      if (it.gitem) pi = (bh * D.G + (it.qrow0 + q)) * D.nch + (it.kt0 / D.chunk_tiles);
+      else orow = bh * n + pos;
 #pragma unroll
-        for (int cc = 0; cc < 4; cc++) w[cc] = lf_range_bits(lo, hi, 32 * cc);
-        if (padded) {
+      for (int hh = 0; hh < 2; hh++) {
+        const int c0 = 32 * g + 16 * hh;
+        uint32_t ra[16], rb[16];
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                     : "=r"(ra[0]), "=r"(ra[1]), "=r"(ra[2]), "=r"(ra[3]), "=r"(ra[4]), "=r"(ra[5]), "=r"(ra[6]), "=r"(ra[7]),
+                       "=r"(ra[8]), "=r"(ra[9]), "=r"(ra[10]), "=r"(ra[11]), "=r"(ra[12]), "=r"(ra[13]), "=r"(ra[14]), "=r"(ra[15])
+                     : "r"(tmem + lane_off + LF_TM_O(0) + c0));
+        if (hasB)
+          asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                       : "=r"(rb[0]), "=r"(rb[1]), "=r"(rb[2]), "=r"(rb[3]), "=r"(rb[4]), "=r"(rb[5]), "=r"(rb[6]), "=r"(rb[7]),
+                         "=r"(rb[8]), "=r"(rb[9]), "=r"(rb[10]), "=r"(rb[11]), "=r"(rb[12]), "=r"(rb[13]), "=r"(rb[14]), "=r"(rb[15])
+                       : "r"(tmem + lane_off + LF_TM_O(1) + c0));
+        asm volatile("tcgen05.wait::ld.sync.aligned;"
+                     : "+r"(ra[0]), "+r"(ra[1]), "+r"(ra[2]), "+r"(ra[3]), "+r"(ra[4]), "+r"(ra[5]), "+r"(ra[6]), "+r"(ra[7]),
+                       "+r"(ra[8]), "+r"(ra[9]), "+r"(ra[10]), "+r"(ra[11]), "+r"(ra[12]), "+r"(ra[13]), "+r"(ra[14]), "+r"(ra[15]),
+                       "+r"(rb[0]), "+r"(rb[1]), "+r"(rb[2]), "+r"(rb[3]), "+r"(rb[4]), "+r"(rb[5]), "+r"(rb[6]), "+r"(rb[7]),
+                       "+r"(rb[8]), "+r"(rb[9]), "+r"(rb[10]), "+r"(rb[11]), "+r"(rb[12]), "+r"(rb[13]), "+r"(rb[14]), "+r"(rb[15])
+                     :
+                     : "memory");
+        float v[16];
 #pragma unroll
-          for (int cc = 0; cc < 4; cc++) {
-            const int tk = kb + 32 * cc + lane;
-            const bool ok = tk >= 0 && tk < cnt && mrow[rho + tk * d] != 0;
-            w[cc] &= __ballot_sync(0xffffffffu, ok);
+        for (int kk = 0; kk < 16; kk++)
+          v[kk] = __uint_as_float(ra[kk]) * ca + (hasB ? __uint_as_float(rb[kk]) * cb : 0.f);
+        if (store_row) {
+          if (it.gitem) {
+            float4 *dst = reinterpret_cast<float4 *>(P.part_acc + pi * LF_HD + c0);
+#pragma unroll
+            for (int kk = 0; kk < 4; kk++)
+              dst[kk] = make_float4(v[4 * kk], v[4 * kk + 1], v[4 * kk + 2], v[4 * kk + 3]);
+          } else {
+            uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(P.o) + orow * LF_HD + c0);
+#pragma unroll
+            for (int kk = 0; kk < 2; kk++) {
+              uint4 u;
+              u.x = lf_pack2<kF16>(v[8 * kk + 0], v[8 * kk + 1]);
+              u.y = lf_pack2<kF16>(v[8 * kk + 2], v[8 * kk + 3]);
+              u.z = lf_pack2<kF16>(v[8 * kk + 4], v[8 * kk + 5]);
+              u.w = lf_pack2<kF16>(v[8 * kk + 6], v[8 * kk + 7]);
+              dst[kk] = u;
+            }
           }
-        }
-      } else {
-        const int gb = (it - nband) * LF_BK;
-        const int hi = active ? min(LF_BK - 1, ng - 1 - gb) : -1;
-#pragma unroll
-        for (int cc = 0; cc < 4; cc++) {
-          uint32_t inwin = lf_range_bits(e_lo - gb, e_hi - 1 - gb, 32 * cc);
-          if (d > 1) {
-            const int e = gb + 32 * cc + lane;
-            const bool res = e < ng && (gl[e] - rho) % d == 0;
-            inwin &= __ballot_sync(0xffffffffu, res);
-          }
-          w[cc] = lf_range_bits(0, hi, 32 * cc) & ~inwin;
         }
       }
-      // ---- probabilities of the tile -> P (TMEM).  Optimistic single pass
-      // against the running reference m_ref; redone (rarely) with the tile's
-      // own max when some row's max grew by more than 2^8.
-      LfPvGate gate{pv_done, it > 0 ? ((it - 1) & 1) : -1, abort_flag, D.status};
-      const bool any_bits = (w[0] | w[1] | w[2] | w[3]) != 0u;
-      const bool single = __all_sync(0xffffffffu, m_ref != -INFINITY || !any_bits);
-      float mx = -INFINITY, lt = 0.f;
-      if (single) lf_softmax_tile<kF16>(tl, w, sl2, m_ref, mx, lt, true, gate);
-      const bool grow = any_bits && (!single || mx * sl2 > m_ref + 8.f);
-      if (__any_sync(0xffffffffu, grow)) {
-        if (!single) {
-          float dummy = 0.f;
-          lf_softmax_tile<kF16>(tl, w, sl2, m_ref, mx, dummy, false, gate);  // max only
-        }
-        const float ms = mx * sl2;
-        const bool need = any_bits && ms > m_ref + 8.f;
-        const float m_new = need ? ms : m_ref;
-        const float alpha = need ? lf_ex2(m_ref - m_new) : 1.f;
-        l *= alpha;
-        if (it > 0 && __any_sync(0xffffffffu, need)) {
-          gate.pass();
-#pragma unroll
-          for (int half = 0; half < 2; half++) {
-            float ov[32];
-            lf_tmem_ld32(tl + LF_TM_O + 32 * half, ov);
-#pragma unroll
-            for (int k = 0; k < 32; k++) ov[k] *= alpha;
-            lf_tmem_st32(tl + LF_TM_O + 32 * half, ov);
-          }
-        }
-        m_ref = m_new;
-        lt = 0.f;
-        float mx2 = -INFINITY;
-        lf_softmax_tile<kF16>(tl, w, sl2, m_ref, mx2, lt, true, gate);
+      if (store_row && g == 0) {
+        if (it.gitem) P.part_ml[pi] = make_float2(M, L);
+        else if (P.lse) P.lse[orow] = code == 1 ? (M + __log2f(L)) * LF_LN2 : -INFINITY;
       }
-      l += lt;
-      gate.pass();  // (no-op unless every chunk of the tile was skipped)
-      lf_tmem_wait_st();
+      // both groups finished reading O before the next item's P.V overwrites it
       lf_tc_fence_before();
       __syncwarp();
-      if (lane == 0) lf_mbar_arrive(p_full);
-    }
-    // ---- epilogue
-    if (alive && lf_wait_warp(o_full, 0, abort_flag, D.status, 9)) {
-      lf_tc_fence_after();
-      float ov[64];
-      {
-        float a[32], c2[32];
-        lf_tmem_ld32(tl + LF_TM_O, a);
-        lf_tmem_ld32(tl + LF_TM_O + 32, c2);
-#pragma unroll
-        for (int k = 0; k < 32; k++) {
-          ov[k] = a[k];
-          ov[32 + k] = c2[k];
-        }
+      if (lane == 0) lf_mbar_arrive(mrg1);
+      if (!lf_wait_warp(mrg1, k & 1, abort_flag, D.status, 13)) {
+        alive = false;
+        break;
       }
-      const size_t bh = (size_t)b * D.H + h;
-      if (gitem) {
-        if (active) {
-          const int e = qrow0 + q;
-          const size_t pi = (bh * D.G + e) * D.nch + (kt0 / D.chunk_tiles);
-          float4 *dst = reinterpret_cast<float4 *>(P.part_acc + pi * LF_HD);
-#pragma unroll
-          for (int k = 0; k < 16; k++)
-            dst[k] = make_float4(ov[4 * k], ov[4 * k + 1], ov[4 * k + 2], ov[4 * k + 3]);
-          P.part_ml[pi] = make_float2(m_ref, l);
-        }
-      } else if (t0 + q < cnt && code != 2) {
-        const size_t orow = bh * n + pos;
-        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(P.o) + orow * LF_HD);
-        const float inv = code == 1 ? 1.f / l : 0.f;
-#pragma unroll
-        for (int k = 0; k < 8; k++) {
-          uint4 v;
-          v.x = lf_pack2<kF16>(ov[8 * k + 0] * inv, ov[8 * k + 1] * inv);
-          v.y = lf_pack2<kF16>(ov[8 * k + 2] * inv, ov[8 * k + 3] * inv);
-          v.z = lf_pack2<kF16>(ov[8 * k + 4] * inv, ov[8 * k + 5] * inv);
-          v.w = lf_pack2<kF16>(ov[8 * k + 6] * inv, ov[8 * k + 7] * inv);
-          dst[k] = v;
-        }
-        if (P.lse) P.lse[orow] = code == 1 ? (m_ref + __log2f(l)) * LF_LN2 : -INFINITY;
-      }
+      k++;
     }
   }
 
   // ---------------------------------------------------- teardown
   lf_tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     lf_tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(LF_TM_COLS)
                  : "memory");
   }
 }
-
 // ------------------------------------------------------------ gather / combine
 
 // Compact, per (b, h), the Q_g rows (global queries) and the K_s / V_s rows
@@ -995,8 +1229,7 @@ int lf_tc_fwd(const LfLaunch &L, const LfTcArgs &a, char *err, size_t errlen) {
   {
     void (*kern)(const LfTcParams) = f16 ? lf_tc_fwd_kernel<1> : lf_tc_fwd_kernel<0>;
     if (!lf_tc_attr_done[f16]) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           LF_SMEM_BYTES);
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LF_SMEM_BYTES);
       if (e != cudaSuccess) {
         snprintf(err, errlen, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         return LF_ERR_CUDA;
@@ -1004,8 +1237,16 @@ int lf_tc_fwd(const LfLaunch &L, const LfTcArgs &a, char *err, size_t errlen) {
       lf_tc_attr_done[f16] = true;
     }
     const long long items = (long long)P.n_gitems + (long long)D.B * P.per_batch;
+    static int nsm = 0;
+    if (nsm == 0) {
+      int dev = 0;
+      cudaGetDevice(&dev);
+      if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
+        nsm = 148;
+    }
+    const unsigned grid = (unsigned)std::min<long long>(items, nsm);  // persistent: one CTA per SM
     if (a.ev_start && a.ev_stop) cudaEventRecord(a.ev_start, L.stream);
-    kern<<<(unsigned)items, LF_TC_THREADS, LF_SMEM_BYTES, L.stream>>>(P);
+    kern<<<grid, LF_TC_THREADS, LF_SMEM_BYTES, L.stream>>>(P);
     lf_launches_add(1);
     if (a.ev_start && a.ev_stop) cudaEventRecord(a.ev_stop, L.stream);
     cudaError_t e = cudaGetLastError();

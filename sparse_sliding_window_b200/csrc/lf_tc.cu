@@ -58,13 +58,13 @@
 #include <utility>
 #include <vector>
 
+#include "lf_ptx.cuh"
 #include "lf_tc.cuh"
 
 #define LF_TC_THREADS 320
 #define LF_TC_NS 5
 #define LF_TC_MAX_MAPS 28
 #define LF_TC_MAX_SEG 32
-#define LF_WAIT_NS 1500000000ull
 
 // TMEM column map (per softmax group g = 0, 1)
 #define LF_TM_S(g) ((g)*128)
@@ -98,409 +98,6 @@ struct LfTcParams {
   float2 *part_ml;
 };
 
-// ------------------------------------------------------------ PTX helpers
-
-__device__ __forceinline__ uint32_t lf_smem(const void *p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ uint64_t lf_globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void lf_mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-
-__device__ __forceinline__ void lf_mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void lf_mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool lf_mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait on an mbarrier phase.  Returns false when the CTA aborted
-// (this thread's own timeout, or another role's).
-__device__ __noinline__ bool lf_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                     int32_t *status, int site) {
-  uint64_t t0 = 0;
-  for (uint32_t it = 0;; it++) {
-    if (lf_mbar_try(bar, parity)) return true;
-    if ((it & 255) == 255) {
-      if (*abort_flag) return false;
-      uint64_t now = lf_globaltimer();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > LF_WAIT_NS) {
-        *abort_flag = 1;
-        lf_set_status(status, LF_ERR_DEVICE_TIMEOUT, site);
-        return false;
-      }
-    }
-  }
-}
-
-// Bounded wait with an inlined first probe (the common, already-complete case).
-__device__ __forceinline__ bool lf_wait_fast(uint32_t bar, uint32_t parity,
-                                             volatile int *abort_flag, int32_t *status, int site) {
-  if (lf_mbar_try(bar, parity)) return true;
-  return lf_wait(bar, parity, abort_flag, status, site);
-}
-
-// Warp-uniform bounded wait: the converged warp polls together (every lane
-// acquires the phase itself), and the verdict is made uniform before the
-// warp-collective tcgen05 instructions that follow.
-__device__ __forceinline__ bool lf_wait_warp(uint32_t bar, uint32_t parity,
-                                             volatile int *abort_flag, int32_t *status, int site) {
-  const bool ok = lf_wait_fast(bar, parity, abort_flag, status, site);
-  return __all_sync(0xffffffffu, ok);
-}
-
-__device__ __forceinline__ void lf_tma_load4(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                             int c0, int c1, int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void lf_tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void lf_tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void lf_tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-
-// D[tmem] (+)= A[smem desc] * B[smem desc]
-__device__ __forceinline__ void lf_mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                          uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem desc]
-__device__ __forceinline__ void lf_mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
-                                          uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-// 32 consecutive fp32 columns of this thread's TMEM lane
-__device__ __forceinline__ void lf_tmem_ld32(uint32_t taddr, float (&x)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int k = 0; k < 32; k++) x[k] = __uint_as_float(r[k]);
-}
-
-__device__ __forceinline__ void lf_tmem_st32(uint32_t taddr, const float (&x)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31, %32};" ::"r"(taddr),
-      "r"(__float_as_uint(x[0])), "r"(__float_as_uint(x[1])), "r"(__float_as_uint(x[2])),
-      "r"(__float_as_uint(x[3])), "r"(__float_as_uint(x[4])), "r"(__float_as_uint(x[5])),
-      "r"(__float_as_uint(x[6])), "r"(__float_as_uint(x[7])), "r"(__float_as_uint(x[8])),
-      "r"(__float_as_uint(x[9])), "r"(__float_as_uint(x[10])), "r"(__float_as_uint(x[11])),
-      "r"(__float_as_uint(x[12])), "r"(__float_as_uint(x[13])), "r"(__float_as_uint(x[14])),
-      "r"(__float_as_uint(x[15])), "r"(__float_as_uint(x[16])), "r"(__float_as_uint(x[17])),
-      "r"(__float_as_uint(x[18])), "r"(__float_as_uint(x[19])), "r"(__float_as_uint(x[20])),
-      "r"(__float_as_uint(x[21])), "r"(__float_as_uint(x[22])), "r"(__float_as_uint(x[23])),
-      "r"(__float_as_uint(x[24])), "r"(__float_as_uint(x[25])), "r"(__float_as_uint(x[26])),
-      "r"(__float_as_uint(x[27])), "r"(__float_as_uint(x[28])), "r"(__float_as_uint(x[29])),
-      "r"(__float_as_uint(x[30])), "r"(__float_as_uint(x[31]))
-      : "memory");
-}
-
-__device__ __forceinline__ void lf_tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
-      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]),
-      "r"(w[15])
-      : "memory");
-}
-
-__device__ __forceinline__ void lf_tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ float lf_ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// two fp32 -> packed bf16x2 / f16x2 (lo = first element), round to nearest even
-template <int kF16>
-__device__ __forceinline__ uint32_t lf_pack2(float lo, float hi) {
-  uint32_t r;
-  if (kF16)
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  else
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 "version 1").
-// start address, leading / stride byte offsets are in 16-byte units.
-__device__ __forceinline__ uint64_t lf_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr & 0x3FFFF) >> 4);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
-}
-
-// Instruction descriptor of kind::f16: fp32 accumulate, A/B bf16 (or f16),
-// M = 128, N = n, A K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1).
-__device__ __forceinline__ uint32_t lf_idesc(int f16, int n, int b_mn) {
-  uint32_t fmt = f16 ? 0u : 1u;
-  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)b_mn << 16) |
-         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-}
-
-// Bits k (0..31) of the 32-column chunk starting at column `base` whose
-// column lies in [lo, hi].
-__device__ __forceinline__ uint32_t lf_range_bits(int lo, int hi, int base) {
-  int a = lo - base, z = hi - base;
-  if (z < 0 || a > 31 || a > z) return 0u;
-  a = max(a, 0);
-  z = min(z, 31);
-  const uint32_t upto = z == 31 ? 0xffffffffu : ((1u << (z + 1)) - 1u);
-  return upto & ~((1u << a) - 1u);
-}
-
-// One pass over the 4 column chunks of a row's S tile (TMEM lane of this
-// thread).  Columns whose bit in w is clear are treated as -inf.  Tracks the
-// row max of the attended raw scores in mx; when write_p, also computes
-// p = 2^(s * sl2 - m) into P (TMEM, packed bf16 / f16) and their sum lt.
-// Chunks no lane of the warp attends are skipped (P written as zeros).
-// TMEM load of 32 columns without waiting; the caller waits with
-// lf_tmem_wait_ld_regs, which also pins the registers behind the wait.
-__device__ __forceinline__ void lf_tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void lf_tmem_wait_ld_regs(uint32_t (&r)[32]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
-                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
-                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
-                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
-                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
-                 "+r"(r[30]), "+r"(r[31])
-               :
-               : "memory");
-}
-
-// packed fp32 pair arithmetic (one instruction for two lanes of data)
-__device__ __forceinline__ uint64_t lf_f2(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void lf_f2_split(uint64_t v, float &a, float &b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ uint64_t lf_fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t lf_add2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
-// Gate before the first write of P (or O) of a tile: the previous P.V of
-// the same softmax group must have finished reading P.  `pending` is the
-// pv_done phase still to be observed, or -1.
-struct LfPvGate {
-  uint32_t bar;
-  int pending;
-  volatile int *abort_flag;
-  int32_t *status;
-  __device__ __forceinline__ bool pass() {
-    if (pending < 0) return true;
-    const bool ok = lf_wait_warp(bar, (uint32_t)pending, abort_flag, status, 10);
-    pending = -1;
-    return ok;
-  }
-};
-
-template <int kF16>
-__device__ __forceinline__ void lf_p_chunk(uint32_t tP, int cc, float (&x)[32], float sl2,
-                                           float mneg, float &lt) {
-  uint32_t pw[16];
-  float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-  for (int k = 0; k < 32; k += 2) {
-    const float p0 = lf_ex2(fmaf(x[k], sl2, mneg));
-    const float p1 = lf_ex2(fmaf(x[k + 1], sl2, mneg));
-    s0 += p0;
-    s1 += p1;
-    pw[k / 2] = lf_pack2<kF16>(p0, p1);
-  }
-  lt += s0 + s1;
-  lf_tmem_st16(tP + 16 * cc, pw);
-}
-
-__device__ __forceinline__ void lf_mask_chunk(float (&x)[32], uint32_t wc) {
-  if (!__all_sync(0xffffffffu, wc == 0xffffffffu)) {
-#pragma unroll
-    for (int k = 0; k < 32; k++) x[k] = ((wc >> k) & 1u) ? x[k] : -INFINITY;
-  }
-}
-
-__device__ __forceinline__ float lf_max32(const float (&x)[32]) {
-  float a = fmaxf(x[0], x[1]), b = fmaxf(x[2], x[3]), c = fmaxf(x[4], x[5]), d = fmaxf(x[6], x[7]);
-#pragma unroll
-  for (int k = 8; k < 32; k += 4) {
-    a = fmaxf(a, x[k]);
-    b = fmaxf(b, x[k + 1]);
-    c = fmaxf(c, x[k + 2]);
-    d = fmaxf(d, x[k + 3]);
-  }
-  return fmaxf(fmaxf(a, b), fmaxf(c, d));
-}
-
-// 64 consecutive fp32 columns of this thread's TMEM lane (one wait)
-__device__ __forceinline__ void lf_tmem_ld32x2(uint32_t taddr, float (&x)[32], float (&y)[32]) {
-  uint32_t r[32], u[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr));
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
-      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
-        "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]),
-        "=r"(u[13]), "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]),
-        "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]),
-        "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]),
-        "=r"(u[31])
-      : "r"(taddr + 32));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int k = 0; k < 32; k++) {
-    x[k] = __uint_as_float(r[k]);
-    y[k] = __uint_as_float(u[k]);
-  }
-}
-
-// One pass over the 4 column chunks of a row's S tile (TMEM lane of this
-// thread).  Columns whose bit in w is clear are treated as -inf.  Tracks the
-// row max of the attended raw scores in mx; when write_p, also computes
-// p = 2^(s * sl2 - m) into P (TMEM, packed bf16 / f16) and their sum lt.
-// Chunks no lane of the warp attends are skipped (P written as zeros); two
-// attended chunks are fetched with one TMEM wait.
-
-template <int kF16>
-__device__ __forceinline__ void lf_softmax_tile(uint32_t tS, uint32_t tP, const uint32_t (&w)[4], float sl2,
-                                                float m, float &mx, float &lt, bool write_p,
-                                                LfPvGate &gate) {
-  const float mneg = m == -INFINITY ? 0.f : -m;
-#pragma unroll
-  for (int pp = 0; pp < 2; pp++) {
-    const int c0 = 2 * pp, c1 = 2 * pp + 1;
-    const bool a0 = __any_sync(0xffffffffu, w[c0] != 0u);
-    const bool a1 = __any_sync(0xffffffffu, w[c1] != 0u);
-    if (write_p && !(a0 && a1)) {
-      gate.pass();
-      uint32_t z[16];
-#pragma unroll
-      for (int k = 0; k < 16; k++) z[k] = 0u;
-      if (!a0) lf_tmem_st16(tP + 16 * c0, z);
-      if (!a1) lf_tmem_st16(tP + 16 * c1, z);
-    }
-    if (a0 && a1) {
-      float x[32], y[32];
-      lf_tmem_ld32x2(tS + 32 * c0, x, y);
-      lf_mask_chunk(x, w[c0]);
-      lf_mask_chunk(y, w[c1]);
-      mx = fmaxf(mx, fmaxf(lf_max32(x), lf_max32(y)));
-      if (write_p) {
-        gate.pass();
-        lf_p_chunk<kF16>(tP, c0, x, sl2, mneg, lt);
-        lf_p_chunk<kF16>(tP, c1, y, sl2, mneg, lt);
-      }
-    } else if (a0 || a1) {
-      const int c = a0 ? c0 : c1;
-      float x[32];
-      lf_tmem_ld32(tS + 32 * c, x);
-      lf_mask_chunk(x, w[c]);
-      mx = fmaxf(mx, lf_max32(x));
-      if (write_p) {
-        gate.pass();
-        lf_p_chunk<kF16>(tP, c, x, sl2, mneg, lt);
-      }
-    }
-  }
-}
 
 // P for one S tile of this thread's TMEM lane against the reference m:
 // p = 2^(s*sl2 - m) for the attended columns (bit set in w), 0 elsewhere,

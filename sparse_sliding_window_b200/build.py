@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "liblf_attn.so")
-SOURCES = ["lf_api.cu", "lf_simt.cu", "lf_tc.cu", "lf_static.cu"]
+SOURCES = ["lf_api.cu", "lf_simt.cu", "lf_tc.cu", "lf_tc_bwd.cu", "lf_static.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -110,17 +110,27 @@ static int lf_prepare(const lf_attn_params *p, int for_bwd, LfDev &dev, LfWs &ws
   off = lf_align(off + B * ((size_t)n + 1) * 4);
   const bool tc = p->dtype != LF_F32 && p->kernel != LF_KERNEL_SIMT;
   ws.qg_c = ws.ks_c = ws.vs_c = ws.part_acc = ws.part_ml = off;
-  if (tc && !for_bwd) {
+  if (tc) {
     ws.qg_c = off;
     off = lf_align(off + B * H * Ga * LF_HD * eb);
     ws.ks_c = off;
     off = lf_align(off + B * H * Gka * LF_HD * eb);
     ws.vs_c = off;
     off = lf_align(off + B * H * Gka * LF_HD * eb);
-    ws.part_acc = off;
-    off = lf_align(off + B * H * Ga * dev.nch * LF_HD * 4);
-    ws.part_ml = off;
-    off = lf_align(off + B * H * Ga * dev.nch * 8);
+    if (!for_bwd) {
+      // split-KV partials of the global rows
+      ws.part_acc = off;
+      off = lf_align(off + B * H * Ga * dev.nch * LF_HD * 4);
+      ws.part_ml = off;
+      off = lf_align(off + B * H * Ga * dev.nch * 8);
+    } else {
+      // backward: per-chunk partials of the global columns (dK, dV) and rows (dQ_g)
+      const size_t nchb = ((size_t)n + 255) / 256;
+      ws.part_acc = off;
+      off = lf_align(off + B * H * Ga * nchb * 2 * LF_HD * 4);
+      ws.part_ml = off;
+      off = lf_align(off + B * H * Ga * nchb * LF_HD * 4);
+    }
   }
   ws.delta = off;
   if (for_bwd) off = lf_align(off + B * H * (size_t)n * 4);
@@ -219,6 +229,12 @@ extern "C" int lf_attn_bwd(const lf_attn_params *p, const void *q_s, const void 
   LfLaunch L;
   if ((st = lf_bind_ws(p, 1, workspace, ws_bytes, mask, stream, L))) return st;
   if ((st = lf_cuda(lf_launch_mask_pass(L), "mask pass"))) return st;
+  if (p->dtype != LF_F32 && p->kernel != LF_KERNEL_SIMT) {
+    LfTcBwdArgs a{q_s, k_s, v_s, q_g, k_g, v_g, o, lse, d_o, dq_s, dk_s, dv_s, dq_g, dk_g, dv_g};
+    st = lf_tc_bwd(L, a, g_err, sizeof(g_err));
+    if (st != LF_ERR_UNSUPPORTED || p->kernel != LF_KERNEL_AUTO) return st;
+    g_err[0] = 0;  // shape outside the tensor-core kernel's parameter block
+  }
   return lf_cuda(lf_launch_simt_bwd(L, q_s, k_s, v_s, q_g, k_g, v_g, o, lse, d_o, dq_s, dk_s, dv_s,
                                     dq_g, dk_g, dv_g),
                  "backward");

@@ -49,7 +49,7 @@ __device__ __forceinline__ bool lf_mbar_try(uint32_t bar, uint32_t parity) {
 
 // Bounded wait on an mbarrier phase.  Returns false when the CTA aborted
 // (this thread's own timeout, or another role's).
-__device__ __noinline__ bool lf_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+static __device__ __noinline__ bool lf_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                      int32_t *status, int site) {
   uint64_t t0 = 0;
   for (uint32_t it = 0;; it++) {

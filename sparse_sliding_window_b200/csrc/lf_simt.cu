@@ -453,3 +453,29 @@ cudaError_t lf_launch_simt_bwd(const LfLaunch &L, const void *qs, const void *ks
                                    dkg, dvg);
   }
 }
+
+// delta = rowsum(dO * O) and dK_g / dV_g (every key, over the global rows),
+// shared by the CUDA-core and the tensor-core backward.
+template <typename T>
+static cudaError_t lf_bwd_delta_dkvg_t(const LfLaunch &L, const void *o, const void *dO,
+                                       float *delta, const void *qg, const void *kg,
+                                       const void *vg, const float *lse, void *dkg, void *dvg) {
+  long long rows = (long long)L.dev.B * L.dev.H * L.dev.n;
+  unsigned grid = (unsigned)((rows + 7) / 8);
+  lf_bwd_delta_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)o, (const T *)dO, delta);
+  lf_bwd_dkv_g_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)qg, (const T *)kg,
+                                                     (const T *)vg, lse, (const T *)dO, delta,
+                                                     (T *)dkg, (T *)dvg);
+  lf_launches_add(2);
+  return cudaGetLastError();
+}
+
+cudaError_t lf_launch_bwd_delta_dkvg(const LfLaunch &L, const void *o, const void *dO, float *delta,
+                                     const void *qg, const void *kg, const void *vg, const float *lse,
+                                     void *dkg, void *dvg) {
+  if (L.dtype == LF_F16)
+    return lf_bwd_delta_dkvg_t<__half>(L, o, dO, delta, qg, kg, vg, lse, dkg, dvg);
+  if (L.dtype == LF_BF16)
+    return lf_bwd_delta_dkvg_t<__nv_bfloat16>(L, o, dO, delta, qg, kg, vg, lse, dkg, dvg);
+  return lf_bwd_delta_dkvg_t<float>(L, o, dO, delta, qg, kg, vg, lse, dkg, dvg);
+}

@@ -81,9 +81,6 @@
 #define LF_SM_XCH (LF_SM_BAR + 512)
 #define LF_SMEM_BYTES (LF_SM_XCH + 2 * LF_BQ * 8)
 
-struct LfTcSeg {
-  int h0, h1, d, rho, cnt, nqb, start, map;
-};
 
 struct LfTcParams {
   CUtensorMap maps[LF_TC_MAX_MAPS];
@@ -719,7 +716,7 @@ static PFN_cuTensorMapEncodeTiled lf_encode_fn() {
 
 // 4-D tiled map over rows of 64 elements: dims {64, rows, H, B}; strides in
 // bytes {row_stride, head_stride, batch_stride}; box {64, box_rows, 1, 1}.
-static bool lf_make_map(CUtensorMap *m, int f16, const void *base, uint64_t rows, uint64_t H,
+bool lf_make_map(CUtensorMap *m, int f16, const void *base, uint64_t rows, uint64_t H,
                         uint64_t B, uint64_t row_stride, uint64_t head_stride,
                         uint64_t batch_stride, uint32_t box_rows) {
   PFN_cuTensorMapEncodeTiled enc = lf_encode_fn();
@@ -733,6 +730,23 @@ static bool lf_make_map(CUtensorMap *m, int f16, const void *base, uint64_t rows
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+cudaError_t lf_launch_gather(const LfLaunch &L, const void *qg, const void *ks, const void *vs,
+                             void *qg_c, void *ks_c, void *vs_c, int Ga, int Gka) {
+  const LfDev &D = L.dev;
+  const long long rows = (long long)D.B * D.H * Gka;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  if (L.dtype == LF_F16)
+    lf_gather_kernel<__half><<<grid, 256, 0, L.stream>>>(D, (const __half *)qg, (const __half *)ks,
+                                                         (const __half *)vs, (__half *)qg_c,
+                                                         (__half *)ks_c, (__half *)vs_c, Ga, Gka);
+  else
+    lf_gather_kernel<__nv_bfloat16><<<grid, 256, 0, L.stream>>>(
+        D, (const __nv_bfloat16 *)qg, (const __nv_bfloat16 *)ks, (const __nv_bfloat16 *)vs,
+        (__nv_bfloat16 *)qg_c, (__nv_bfloat16 *)ks_c, (__nv_bfloat16 *)vs_c, Ga, Gka);
+  lf_launches_add(1);
+  return cudaGetLastError();
 }
 
 static bool lf_tc_attr_done[2] = {false, false};
@@ -809,18 +823,11 @@ int lf_tc_fwd(const LfLaunch &L, const LfTcArgs &a, char *err, size_t errlen) {
     P.part_ml = (float2 *)(L.ws_base + L.ws.part_ml);
     (void)eb;
     if (G > 0) {
-      const long long rows = (long long)D.B * D.H * Gka;
-      const unsigned grid = (unsigned)((rows + 7) / 8);
-      if (f16)
-        lf_gather_kernel<__half><<<grid, 256, 0, L.stream>>>(
-            D, (const __half *)a.qg, (const __half *)a.ks, (const __half *)a.vs, (__half *)qg_c,
-            (__half *)ks_c, (__half *)vs_c, Ga, Gka);
-      else
-        lf_gather_kernel<__nv_bfloat16><<<grid, 256, 0, L.stream>>>(
-            D, (const __nv_bfloat16 *)a.qg, (const __nv_bfloat16 *)a.ks,
-            (const __nv_bfloat16 *)a.vs, (__nv_bfloat16 *)qg_c, (__nv_bfloat16 *)ks_c,
-            (__nv_bfloat16 *)vs_c, Ga, Gka);
-      lf_launches_add(1);
+      cudaError_t e = lf_launch_gather(L, a.qg, a.ks, a.vs, qg_c, ks_c, vs_c, Ga, Gka);
+      if (e != cudaSuccess) {
+        snprintf(err, errlen, "gather launch: %s", cudaGetErrorString(e));
+        return LF_ERR_CUDA;
+      }
     }
   }
   {

@@ -1,0 +1,730 @@
+// lf_tc_bwd.cu -- tensor-core (tcgen05 / TMEM / TMA) backward of Longformer
+// attention, bf16 / f16 inputs, fp32 accumulation, for the loss L = sum(o * dO).
+//
+// With P the attention probabilities (recomputed from the forward's
+// log-normaliser, never stored), dP = dO V^T, D_i = rowsum(dO_i * O_i) and
+// dS = P * (dP - D) * scale:   dQ = dS K,  dK = dS^T Q,  dV = P^T dO
+// (the softmax Jacobian; global rows use Q_g / K_g / V_g, local rows
+// Q_s / K_s / V_s, segmentfault page sections 全局注意力 / 全局注意力的线性投影).
+//
+// Two work-item kinds run on the same tensor-core pipeline, one 128-row
+// block of a residue sub-sequence per CTA (dilated heads use the forward's
+// residue tensor-map views):
+//  * mode Q  (rows = local queries):  per key tile  S = Q K^T, dP = dO V^T;
+//             the softmax warps form dS (TMEM) and the MMA warp accumulates
+//             dQ += dS K.  Key tiles are the band tiles of the block and the
+//             global-column tiles (global keys outside each row's window).
+//             Writes dQ_s (zero for global and mask-0 rows).
+//  * mode KV (rows = keys):  per band query tile  S^T = K Q^T, dP^T = V dO^T;
+//             the softmax warps form P^T and dS^T (TMEM) from the queries'
+//             log-normaliser and D (staged per tile in shared memory by the
+//             producer warp; +inf log-normaliser for columns that are not
+//             local queries, so their probability is 0), and the MMA warp
+//             accumulates dV += P^T dO, dK += dS^T Q.  Writes the band part of
+//             dK_s, dV_s (the global-column part of the global keys is added
+//             afterwards by lf_bwd_gcol_*).
+// Roles per CTA (192 threads, one CTA per SM: all 512 TMEM columns): warps
+// 0-3 form P / dS (one TMEM lane = one row), warp 4 issues TMA loads (row
+// operands once, column operands into a 3-stage ring), warp 5 issues the
+// MMAs.  TMEM: S [0,128), dP [128,256), acc0 [256,320) (dQ or dV),
+// acc1 [320,384) (dK), A0 [384,448) (dS or P^T), A1 [448,512) (dS^T).
+// Every mbarrier wait is bounded (status LF_ERR_DEVICE_TIMEOUT on expiry).
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <map>
+#include <utility>
+
+#include "lf_ptx.cuh"
+#include "lf_tc.cuh"
+
+#define LF_BW_THREADS 192
+#define LF_BW_NS 3
+#define LF_BW_MAX_MAPS 40
+#define LF_BW_MAX_SEG 32
+#define LF_BW_ROWS_PER_CHUNK 256  // rows (keys) per warp of the global-row / -column parts
+
+#define LF_BW_R0 0
+#define LF_BW_R1 16384
+#define LF_BW_C0(s) (32768 + (s)*32768)
+#define LF_BW_C1(s) (32768 + (s)*32768 + 16384)
+#define LF_BW_VEC(s) (32768 + LF_BW_NS * 32768 + (s)*1024)
+#define LF_BW_BAR (32768 + LF_BW_NS * 32768 + LF_BW_NS * 1024)
+#define LF_BW_SMEM (LF_BW_BAR + 256)
+
+#define LF_BT_S 0
+#define LF_BT_DP 128
+#define LF_BT_ACC0 256
+#define LF_BT_ACC1 320
+#define LF_BT_A0 384
+#define LF_BT_A1 448
+
+struct LfBwParams {
+  CUtensorMap maps[LF_BW_MAX_MAPS];  // per residue view: q, k, v, dO; then ks_c, vs_c
+  LfDev dev;
+  LfTcSeg seg[LF_BW_MAX_SEG];
+  int nseg, per_batch, gbox, map_ksc, map_vsc;
+  const float *lse;
+  const float *delta;
+  void *out0;  // dQ_s (mode Q) or dV_s (mode KV)
+  void *out1;  // dK_s (mode KV)
+};
+
+// Work item (shared decode for every role).
+struct LfBwItem {
+  int b, h, d, rho, cnt, row0, map, nband, nglob, T, ng;
+};
+
+__device__ __forceinline__ void lf_bw_decode(const LfBwParams &P, int idx, int modeq,
+                                             LfBwItem &it) {
+  const LfDev &D = P.dev;
+  it.b = idx / P.per_batch;
+  int rem = idx - it.b * P.per_batch;
+  int s = 0;
+  while (s + 1 < P.nseg && rem >= P.seg[s + 1].start) s++;
+  const LfTcSeg &sg = P.seg[s];
+  rem -= sg.start;
+  it.h = sg.h0 + rem / sg.nqb;
+  it.row0 = (rem % sg.nqb) * LF_BQ;
+  it.d = sg.d;
+  it.rho = sg.rho;
+  it.cnt = sg.cnt;
+  it.map = sg.map;
+  it.nband = lf_band_tiles(D.r, D.causal);
+  const int32_t *bi = D.binfo + (size_t)it.b * LF_BI_WORDS;
+  it.ng = bi[LF_BI_NG];
+  it.nglob = 0;
+  if (modeq && it.ng > 0) {
+    bool need = true;
+    if (it.d == 1 && !D.causal) {
+      const int tlast = min(it.row0 + LF_BQ - 1, it.cnt - 1);
+      if (bi[LF_BI_GMIN] >= tlast - D.r && bi[LF_BI_GMAX] <= it.row0 + D.r) need = false;
+    }
+    it.nglob = need ? (it.ng + LF_BK - 1) / LF_BK : 0;
+  }
+  it.T = it.nband + it.nglob;
+}
+
+// first column-operand row of band tile u
+__device__ __forceinline__ int lf_bw_tile_row(const LfDev &D, const LfBwItem &it, int modeq, int u) {
+  if (modeq || !D.causal) return it.row0 - D.r + LF_BK * u;
+  return it.row0 + LF_BK * u;  // causal, rows = keys: queries t in [j, j + r]
+}
+
+template <int kF16, int kModeQ>
+__global__ void __launch_bounds__(LF_BW_THREADS, 1)
+    lf_tc_bwd_kernel(const __grid_constant__ LfBwParams P) {
+  extern __shared__ __align__(1024) uint8_t lf_bw_smem[];
+  const uint32_t sbase = lf_smem(lf_bw_smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) lf_set_status(P.dev.status, LF_ERR_UNSUPPORTED, 9001);
+    return;
+  }
+  uint8_t *gbase = lf_bw_smem;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const LfDev &D = P.dev;
+  const int n = D.n;
+  LfBwItem it;
+  lf_bw_decode(P, blockIdx.x, kModeQ, it);
+  const int T = it.T;
+
+  const uint32_t bar = sbase + LF_BW_BAR;
+  const uint32_t row_full = bar, s_full = bar + 8, ds_full = bar + 16, acc_done = bar + 24,
+                 o_full = bar + 32, end_bar = bar + 40;
+  const uint32_t col_full0 = bar + 48, col_empty0 = bar + 48 + 8 * LF_BW_NS;
+  uint32_t *tmem_slot = (uint32_t *)(gbase + LF_BW_BAR + 192);
+  volatile int *abort_flag = (volatile int *)(gbase + LF_BW_BAR + 196);
+
+  if (threadIdx.x == 0) {
+    lf_mbar_init(row_full, 1);
+    lf_mbar_init(s_full, 1);
+    lf_mbar_init(ds_full, 4);
+    lf_mbar_init(acc_done, 1);
+    lf_mbar_init(o_full, 1);
+    lf_mbar_init(end_bar, 1);
+    for (int s = 0; s < LF_BW_NS; s++) {
+      lf_mbar_init(col_full0 + 8 * s, kModeQ ? 1 : 2);
+      lf_mbar_init(col_empty0 + 8 * s, 1);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 5) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     lf_smem(tmem_slot)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  lf_tc_fence_before();
+  __syncthreads();
+  lf_tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const size_t bh = (size_t)it.b * D.H + it.h;
+  const int32_t *mrow = D.mask + (size_t)it.b * n;
+
+  if (warp == 4) {
+    // ================================================== TMA producer (+ column vectors)
+    const CUtensorMap *mq = &P.maps[it.map], *mk = &P.maps[it.map + 1], *mv = &P.maps[it.map + 2],
+                      *mdo = &P.maps[it.map + 3];
+    if (lane == 0) {
+      lf_mbar_expect_tx(row_full, 32768);
+      lf_tma_load4(sbase + LF_BW_R0, kModeQ ? mq : mk, row_full, 0, it.row0, it.h, it.b);
+      lf_tma_load4(sbase + LF_BW_R1, kModeQ ? mdo : mv, row_full, 0, it.row0, it.h, it.b);
+    }
+    int issued = 0;
+    for (int t = 0; t < T; t++) {
+      const int s = t % LF_BW_NS;
+      if (t >= LF_BW_NS &&
+          !lf_wait_warp(col_empty0 + 8 * s, ((t / LF_BW_NS) & 1) ^ 1, abort_flag, D.status, 21))
+        break;
+      int row;
+      const CUtensorMap *c0, *c1;
+      uint32_t bytes;
+      if (t < it.nband) {
+        row = lf_bw_tile_row(D, it, kModeQ, t);
+        c0 = kModeQ ? mk : mq;
+        c1 = kModeQ ? mv : mdo;
+        bytes = 32768;
+      } else {
+        row = (t - it.nband) * LF_BK;
+        c0 = &P.maps[P.map_ksc];
+        c1 = &P.maps[P.map_vsc];
+        bytes = 2 * P.gbox * 128;
+      }
+      if (!kModeQ) {
+        // per-column (query) log-normaliser in log2 units and D; +inf marks
+        // columns that are not local queries (probability 0)
+        float *lse2 = (float *)(gbase + LF_BW_VEC(s));
+        float *dv = lse2 + LF_BQ;
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          const int c = lane + 32 * k, tq = row + c;
+          float l2 = INFINITY, dd = 0.f;
+          if (tq >= 0 && tq < it.cnt) {
+            const int pos = it.rho + tq * it.d;
+            if (mrow[pos] == 1) {
+              l2 = P.lse[bh * n + pos] * LF_LOG2E;
+              dd = P.delta[bh * n + pos];
+            }
+          }
+          lse2[c] = l2;
+          dv[c] = dd;
+        }
+        __syncwarp();
+      }
+      if (lane == 0) {
+        lf_mbar_expect_tx(col_full0 + 8 * s, bytes);
+        lf_tma_load4(sbase + LF_BW_C0(s), c0, col_full0 + 8 * s, 0, row, it.h, it.b);
+        lf_tma_load4(sbase + LF_BW_C1(s), c1, col_full0 + 8 * s, 0, row, it.h, it.b);
+        if (!kModeQ) lf_mbar_arrive(col_full0 + 8 * s);
+      }
+      issued = t + 1;
+    }
+    if (*abort_flag && lane == 0) {
+      for (int t = max(0, issued - LF_BW_NS); t < issued; t++)
+        lf_wait(col_full0 + 8 * (t % LF_BW_NS), (t / LF_BW_NS) & 1, abort_flag, D.status, 22);
+    }
+  } else if (warp == 5) {
+    // ================================================== MMA issuer
+    if (lane == 0) {
+      const uint64_t dr0 = lf_sdesc(sbase + LF_BW_R0, 16, 1024);
+      const uint64_t dr1 = lf_sdesc(sbase + LF_BW_R1, 16, 1024);
+      const uint64_t dc0 = lf_sdesc(sbase + LF_BW_C0(0), 16, 1024);  // K-major view
+      const uint64_t dc0mn = lf_sdesc(sbase + LF_BW_C0(0), 0, 1024);  // MN-major view
+      const uint64_t dc1 = lf_sdesc(sbase + LF_BW_C1(0), 16, 1024);
+      const uint64_t dc1mn = lf_sdesc(sbase + LF_BW_C1(0), 0, 1024);
+      const uint32_t id_acc = lf_idesc(kF16, 64, 1);
+      const int ngk = (it.ng + 15) / 16 * 16;
+      auto ncols = [&](int t) { return t < it.nband ? LF_BK : min(LF_BK, ngk - (t - it.nband) * LF_BK); };
+      auto issue_s = [&](int t) {
+        const uint64_t so = (uint64_t)((t % LF_BW_NS) * (32768 >> 4));
+        const uint32_t id = lf_idesc(kF16, ncols(t), 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++) {
+          lf_mma_ss(tmem + LF_BT_S, dr0 + 2 * kk, dc0 + so + 2 * kk, id, kk > 0);
+          lf_mma_ss(tmem + LF_BT_DP, dr1 + 2 * kk, dc1 + so + 2 * kk, id, kk > 0);
+        }
+      };
+      bool ok = lf_wait_fast(row_full, 0, abort_flag, D.status, 23) &&
+                lf_wait_fast(col_full0, 0, abort_flag, D.status, 24);
+      if (ok) {
+        lf_tc_fence_after();
+        issue_s(0);
+        lf_tc_commit(s_full);
+        for (int t = 0; t < T; t++) {
+          if (!lf_wait_fast(ds_full, t & 1, abort_flag, D.status, 25)) break;
+          lf_tc_fence_after();
+          if (t + 1 < T) {
+            const int s2 = (t + 1) % LF_BW_NS;
+            if (!lf_wait_fast(col_full0 + 8 * s2, ((t + 1) / LF_BW_NS) & 1, abort_flag, D.status, 26))
+              break;
+            lf_tc_fence_after();
+            issue_s(t + 1);
+            lf_tc_commit(s_full);
+          }
+          const uint64_t so = (uint64_t)((t % LF_BW_NS) * (32768 >> 4));
+          const int ksteps = ncols(t) / 16;
+#pragma unroll
+          for (int kk = 0; kk < 8; kk++) {
+            if (kk >= ksteps) continue;
+            const uint32_t acc = (t > 0 || kk > 0);
+            if (kModeQ) {
+              // dQ += dS K   (K tile as the MN-major B operand)
+              lf_mma_ts(tmem + LF_BT_ACC0, tmem + LF_BT_A0 + 8 * kk, dc0mn + so + 128 * kk, id_acc, acc);
+            } else {
+              // dV += P^T dO ; dK += dS^T Q
+              lf_mma_ts(tmem + LF_BT_ACC0, tmem + LF_BT_A0 + 8 * kk, dc1mn + so + 128 * kk, id_acc, acc);
+              lf_mma_ts(tmem + LF_BT_ACC1, tmem + LF_BT_A1 + 8 * kk, dc0mn + so + 128 * kk, id_acc, acc);
+            }
+          }
+          lf_tc_commit(col_empty0 + 8 * (t % LF_BW_NS));
+          lf_tc_commit(acc_done);
+          if (t + 1 == T) lf_tc_commit(o_full);
+        }
+      }
+      lf_tc_commit(end_bar);
+      lf_wait(end_bar, 0, abort_flag, D.status, 27);
+    }
+  } else {
+    // ================================================== P / dS warps (0..3)
+    const int q = warp * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off + LF_BT_S, tDP = tmem + lane_off + LF_BT_DP;
+    const uint32_t tA0 = tmem + lane_off + LF_BT_A0, tA1 = tmem + lane_off + LF_BT_A1;
+    const float sl2 = D.scale_log2, scale = D.scale;
+    const int trow = it.row0 + q;
+    int pos = 0, code = 0;
+    if (trow < it.cnt) {
+      pos = it.rho + trow * it.d;
+      code = mrow[pos];
+    }
+    // mode Q: local query rows; mode KV: valid key rows
+    const bool active = kModeQ ? (code == 1) : (trow < it.cnt && code != 0);
+    float lse2 = 0.f, dd = 0.f;
+    if (kModeQ && active) {
+      lse2 = P.lse[bh * n + pos] * LF_LOG2E;
+      dd = P.delta[bh * n + pos];
+    }
+    const bool padded = D.binfo[(size_t)it.b * LF_BI_WORDS + LF_BI_NVALID] < n;
+    const int32_t *gl = D.gidx + (size_t)it.b * D.G;
+    int e_lo = 0, e_hi = 0;
+    if (kModeQ && it.nglob > 0 && active) {
+      const int32_t *gr = D.grank + (size_t)it.b * (n + 1);
+      e_lo = gr[max(pos - D.r * it.d, 0)];
+      e_hi = gr[min((D.causal ? pos : pos + D.r * it.d) + 1, n)];
+    }
+    bool alive = true;
+    for (int t = 0; t < T && alive; t++) {
+      if (!lf_wait_warp(s_full, t & 1, abort_flag, D.status, 28)) {
+        alive = false;
+        break;
+      }
+      lf_tc_fence_after();
+      uint32_t w[4];
+      const int s = t % LF_BW_NS;
+      if (t < it.nband) {
+        const int kb = lf_bw_tile_row(D, it, kModeQ, t);
+        int lo, hi;
+        lf_band_cols(q, t, D.r, D.causal, lo, hi);
+        lo = max(lo, -kb);  // column operand rows exist on [0, cnt)
+        hi = min(hi, it.cnt - 1 - kb);
+        if (!active) hi = -1;
+#pragma unroll
+        for (int cc = 0; cc < 4; cc++) w[cc] = lf_range_bits(lo, hi, 32 * cc);
+        if (kModeQ && padded) {
+#pragma unroll
+          for (int cc = 0; cc < 4; cc++) {
+            const int tk = kb + 32 * cc + lane;
+            const bool okk = tk >= 0 && tk < it.cnt && mrow[it.rho + tk * it.d] != 0;
+            w[cc] &= __ballot_sync(0xffffffffu, okk);
+          }
+        }
+      } else {
+        const int gbs = (t - it.nband) * LF_BK;
+        const int hi = active ? min(LF_BK - 1, it.ng - 1 - gbs) : -1;
+#pragma unroll
+        for (int cc = 0; cc < 4; cc++) {
+          uint32_t inwin = lf_range_bits(e_lo - gbs, e_hi - 1 - gbs, 32 * cc);
+          if (it.d > 1) {
+            const int e = gbs + 32 * cc + lane;
+            const bool res = e < it.ng && (gl[e] - it.rho) % it.d == 0;
+            inwin &= __ballot_sync(0xffffffffu, res);
+          }
+          w[cc] = lf_range_bits(0, hi, 32 * cc) & ~inwin;
+        }
+      }
+      if (!kModeQ) {
+        // the per-column vectors of stage s were written by the producer
+        // warp before it arrived on col_full(s): observe that phase here too
+        if (!lf_wait_warp(col_full0 + 8 * s, (t / LF_BW_NS) & 1, abort_flag, D.status, 31)) {
+          alive = false;
+          break;
+        }
+      }
+      const float *clse2 = (const float *)(gbase + LF_BW_VEC(s));
+      const float *cdd = clse2 + LF_BQ;
+      bool gated = (t == 0);
+#pragma unroll
+      for (int cc = 0; cc < 4; cc++) {
+        uint32_t ds_w[16], p_w[16];
+        if (__any_sync(0xffffffffu, w[cc] != 0u)) {
+          float x[32], y[32];
+          lf_tmem_ld32(tS + 32 * cc, x);
+          lf_tmem_ld32(tDP + 32 * cc, y);
+          const uint32_t wc = w[cc];
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            float p0 = 0.f, p1 = 0.f, g0 = 0.f, g1 = 0.f;
+            const float l0 = kModeQ ? lse2 : clse2[32 * cc + k];
+            const float l1 = kModeQ ? lse2 : clse2[32 * cc + k + 1];
+            const float d0 = kModeQ ? dd : cdd[32 * cc + k];
+            const float d1 = kModeQ ? dd : cdd[32 * cc + k + 1];
+            if ((wc >> k) & 1u) {
+              p0 = lf_ex2(fmaf(x[k], sl2, -l0));
+              g0 = p0 * (y[k] - d0) * scale;
+            }
+            if ((wc >> (k + 1)) & 1u) {
+              p1 = lf_ex2(fmaf(x[k + 1], sl2, -l1));
+              g1 = p1 * (y[k + 1] - d1) * scale;
+            }
+            ds_w[k / 2] = lf_pack2<kF16>(g0, g1);
+            p_w[k / 2] = lf_pack2<kF16>(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; k++) ds_w[k] = p_w[k] = 0u;
+        }
+        if (!gated) {
+          // the previous tile's accumulate MMAs have finished reading A0 / A1
+          if (!lf_wait_warp(acc_done, (t - 1) & 1, abort_flag, D.status, 29)) {
+            alive = false;
+            break;
+          }
+          gated = true;
+        }
+        if (kModeQ) {
+          lf_tmem_st16(tA0 + 16 * cc, ds_w);
+        } else {
+          lf_tmem_st16(tA0 + 16 * cc, p_w);
+          lf_tmem_st16(tA1 + 16 * cc, ds_w);
+        }
+      }
+      if (!alive) break;
+      lf_tmem_wait_st();
+      lf_tc_fence_before();
+      __syncwarp();
+      if (lane == 0) lf_mbar_arrive(ds_full);
+    }
+    // ---- epilogue: accumulators -> gradient rows
+    if (alive && lf_wait_warp(o_full, 0, abort_flag, D.status, 30)) {
+      lf_tc_fence_after();
+      if (trow < it.cnt) {
+        const size_t orow = bh * n + pos;
+#pragma unroll
+        for (int which = 0; which < (kModeQ ? 1 : 2); which++) {
+          float a[32], c2[32];
+          lf_tmem_ld32(tmem + lane_off + (which ? LF_BT_ACC1 : LF_BT_ACC0), a);
+          lf_tmem_ld32(tmem + lane_off + (which ? LF_BT_ACC1 : LF_BT_ACC0) + 32, c2);
+          const float keep = active ? 1.f : 0.f;
+          void *outp = which ? P.out1 : P.out0;
+          uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(outp) + orow * LF_HD);
+#pragma unroll
+          for (int k = 0; k < 4; k++) {
+            uint4 u;
+            u.x = lf_pack2<kF16>(a[8 * k + 0] * keep, a[8 * k + 1] * keep);
+            u.y = lf_pack2<kF16>(a[8 * k + 2] * keep, a[8 * k + 3] * keep);
+            u.z = lf_pack2<kF16>(a[8 * k + 4] * keep, a[8 * k + 5] * keep);
+            u.w = lf_pack2<kF16>(a[8 * k + 6] * keep, a[8 * k + 7] * keep);
+            dst[k] = u;
+            uint4 v;
+            v.x = lf_pack2<kF16>(c2[8 * k + 0] * keep, c2[8 * k + 1] * keep);
+            v.y = lf_pack2<kF16>(c2[8 * k + 2] * keep, c2[8 * k + 3] * keep);
+            v.z = lf_pack2<kF16>(c2[8 * k + 4] * keep, c2[8 * k + 5] * keep);
+            v.w = lf_pack2<kF16>(c2[8 * k + 6] * keep, c2[8 * k + 7] * keep);
+            dst[4 + k] = v;
+          }
+        }
+      }
+    }
+  }
+
+  lf_tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    lf_tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                 : "memory");
+  }
+}
+
+// ============================================== global-token parts (CUDA cores)
+
+// Global-column part of dK_s / dV_s: a global key g is attended by every
+// local row, by its window or by its global column (union); the band kernel
+// covered the window, this pass the rows whose window misses g.  One warp per
+// (b, h, global e, chunk of rows); partial sums, reduced by lf_bwd_gcol_reduce.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    lf_bwd_gcol_kernel(LfDev P, const T *qs, const T *ks, const T *vs, const float *lse,
+                       const T *dO, const float *delta, float *part, int nch) {
+  const int lane = threadIdx.x & 31;
+  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (w >= (long long)P.B * P.H * P.G * nch) return;
+  const int c = (int)(w % nch);
+  const long long be = w / nch;
+  const int e = (int)(be % P.G);
+  const long long bh = be / P.G;
+  const int h = (int)(bh % P.H), b = (int)(bh / P.H), d = P.dil[h], n = P.n;
+  const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
+  float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+  if (e < ng) {
+    const int g = P.gidx[(size_t)b * P.G + e];
+    const int32_t *m = P.mask + (size_t)b * n;
+    const size_t base = (size_t)bh * n * LF_HD + 2 * lane;
+    const float2 kk = LfIo<T>::ld2(ks + base + (size_t)g * LF_HD);
+    const float2 vv = LfIo<T>::ld2(vs + base + (size_t)g * LF_HD);
+    const int i1 = min(n, (c + 1) * LF_BW_ROWS_PER_CHUNK);
+    for (int i = c * LF_BW_ROWS_PER_CHUNK; i < i1; i++) {
+      if (m[i] != 1 || lf_in_window(i, g, P.r, d, P.causal)) continue;
+      const size_t ioff = base + (size_t)i * LF_HD, ir = (size_t)bh * n + i;
+      const float2 q = LfIo<T>::ld2(qs + ioff), go = LfIo<T>::ld2(dO + ioff);
+      const float2 sd = lf_warp_sum2(q.x * kk.x + q.y * kk.y, go.x * vv.x + go.y * vv.y);
+      const float pr = exp2f(sd.x * P.scale_log2 - lse[ir] * LF_LOG2E);
+      const float ds = pr * (sd.y - delta[ir]) * P.scale;
+      k0 += ds * q.x;
+      k1 += ds * q.y;
+      v0 += pr * go.x;
+      v1 += pr * go.y;
+    }
+  }
+  float *dst = part + ((size_t)be * nch + c) * 2 * LF_HD + 2 * lane;
+  *reinterpret_cast<float2 *>(dst) = make_float2(k0, k1);
+  *reinterpret_cast<float2 *>(dst + LF_HD) = make_float2(v0, v1);
+}
+
+// dK_s[g] += sum of chunks; dV_s[g] likewise (one warp per (b, h, e)).
+template <typename T>
+__global__ void __launch_bounds__(256)
+    lf_bwd_gcol_reduce(LfDev P, const float *part, int nch, T *dks, T *dvs) {
+  const int lane = threadIdx.x & 31;
+  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (w >= (long long)P.B * P.H * P.G) return;
+  const int e = (int)(w % P.G);
+  const long long bh = w / P.G;
+  const int b = (int)(bh / P.H);
+  if (e >= P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG]) return;
+  float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+  for (int c = 0; c < nch; c++) {
+    const float *src = part + ((size_t)w * nch + c) * 2 * LF_HD + 2 * lane;
+    const float2 a = *reinterpret_cast<const float2 *>(src);
+    const float2 v = *reinterpret_cast<const float2 *>(src + LF_HD);
+    k0 += a.x;
+    k1 += a.y;
+    v0 += v.x;
+    v1 += v.y;
+  }
+  const int g = P.gidx[(size_t)b * P.G + e];
+  const size_t off = ((size_t)bh * P.n + g) * LF_HD + 2 * lane;
+  const float2 kb = LfIo<T>::ld2(dks + off), vb = LfIo<T>::ld2(dvs + off);
+  LfIo<T>::st2(dks + off, kb.x + k0, kb.y + k1);
+  LfIo<T>::st2(dvs + off, vb.x + v0, vb.y + v1);
+}
+
+// dQ_g of the global rows: every valid key through Q_g / K_g / V_g.  One warp
+// per (b, h, global e, chunk of keys); partial sums reduced below.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    lf_bwd_grow_kernel(LfDev P, const T *qg, const T *kg, const T *vg, const float *lse,
+                       const T *dO, const float *delta, float *part, int nch) {
+  const int lane = threadIdx.x & 31;
+  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (w >= (long long)P.B * P.H * P.G * nch) return;
+  const int c = (int)(w % nch);
+  const long long be = w / nch;
+  const int e = (int)(be % P.G);
+  const long long bh = be / P.G;
+  const int b = (int)(bh / P.H), n = P.n;
+  const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
+  float a0 = 0.f, a1 = 0.f;
+  if (e < ng) {
+    const int g = P.gidx[(size_t)b * P.G + e];
+    const int32_t *m = P.mask + (size_t)b * n;
+    const size_t base = (size_t)bh * n * LF_HD + 2 * lane;
+    const size_t gr = (size_t)bh * n + g;
+    const float2 q = LfIo<T>::ld2(qg + base + (size_t)g * LF_HD);
+    const float2 go = LfIo<T>::ld2(dO + base + (size_t)g * LF_HD);
+    const float L2 = lse[gr] * LF_LOG2E, Dg = delta[gr];
+    const int j1 = min(n, (c + 1) * LF_BW_ROWS_PER_CHUNK);
+    for (int j = c * LF_BW_ROWS_PER_CHUNK; j < j1; j++) {
+      if (m[j] == 0) continue;
+      const size_t joff = base + (size_t)j * LF_HD;
+      const float2 k = LfIo<T>::ld2(kg + joff), v = LfIo<T>::ld2(vg + joff);
+      const float2 sd = lf_warp_sum2(q.x * k.x + q.y * k.y, go.x * v.x + go.y * v.y);
+      const float pr = exp2f(sd.x * P.scale_log2 - L2);
+      const float ds = pr * (sd.y - Dg) * P.scale;
+      a0 += ds * k.x;
+      a1 += ds * k.y;
+    }
+  }
+  *reinterpret_cast<float2 *>(part + ((size_t)be * nch + c) * LF_HD + 2 * lane) = make_float2(a0, a1);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+    lf_bwd_grow_reduce(LfDev P, const float *part, int nch, T *dqg) {
+  const int lane = threadIdx.x & 31;
+  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (w >= (long long)P.B * P.H * P.G) return;
+  const int e = (int)(w % P.G);
+  const long long bh = w / P.G;
+  const int b = (int)(bh / P.H);
+  if (e >= P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG]) return;
+  float a0 = 0.f, a1 = 0.f;
+  for (int c = 0; c < nch; c++) {
+    const float2 a = *reinterpret_cast<const float2 *>(part + ((size_t)w * nch + c) * LF_HD + 2 * lane);
+    a0 += a.x;
+    a1 += a.y;
+  }
+  const int g = P.gidx[(size_t)b * P.G + e];
+  LfIo<T>::st2(dqg + ((size_t)bh * P.n + g) * LF_HD + 2 * lane, a0, a1);
+}
+
+// ============================================== host
+
+template <typename T>
+static cudaError_t lf_bwd_global_parts(const LfLaunch &L, const LfTcBwdArgs &a, const float *delta,
+                                       float *part_kv, float *part_q, int nch) {
+  const LfDev &D = L.dev;
+  cudaError_t e;
+  // dQ_g: zero rows outside the global tokens, then the global rows
+  e = cudaMemsetAsync(a.dqg, 0, (size_t)D.B * D.H * D.n * LF_HD * sizeof(T), L.stream);
+  if (e != cudaSuccess) return e;
+  if (D.G > 0) {
+    const long long wk = (long long)D.B * D.H * D.G * nch, wr = (long long)D.B * D.H * D.G;
+    lf_bwd_gcol_kernel<T><<<(unsigned)((wk + 7) / 8), 256, 0, L.stream>>>(
+        D, (const T *)a.qs, (const T *)a.ks, (const T *)a.vs, a.lse, (const T *)a.dO, delta, part_kv, nch);
+    lf_bwd_gcol_reduce<T><<<(unsigned)((wr + 7) / 8), 256, 0, L.stream>>>(D, part_kv, nch, (T *)a.dks,
+                                                                           (T *)a.dvs);
+    lf_bwd_grow_kernel<T><<<(unsigned)((wk + 7) / 8), 256, 0, L.stream>>>(
+        D, (const T *)a.qg, (const T *)a.kg, (const T *)a.vg, a.lse, (const T *)a.dO, delta, part_q, nch);
+    lf_bwd_grow_reduce<T><<<(unsigned)((wr + 7) / 8), 256, 0, L.stream>>>(D, part_q, nch, (T *)a.dqg);
+    lf_launches_add(4);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t lf_launch_bwd_delta_dkvg(const LfLaunch &L, const void *o, const void *dO, float *delta,
+                                     const void *qg, const void *kg, const void *vg, const float *lse,
+                                     void *dkg, void *dvg);
+
+int lf_tc_bwd(const LfLaunch &L, const LfTcBwdArgs &a, char *err, size_t errlen) {
+  const LfDev &D = L.dev;
+  const int f16 = L.dtype == LF_F16 ? 1 : 0;
+  float *delta = (float *)(L.ws_base + L.ws.delta);
+  cudaError_t ce;
+  // delta = rowsum(dO * O); dK_g, dV_g (every key, over the global rows)
+  ce = lf_launch_bwd_delta_dkvg(L, a.o, a.dO, delta, a.qg, a.kg, a.vg, a.lse, a.dkg, a.dvg);
+  if (ce != cudaSuccess) {
+    snprintf(err, errlen, "backward delta / dK_g launch: %s", cudaGetErrorString(ce));
+    return LF_ERR_CUDA;
+  }
+  LfBwParams P;
+  memset(&P, 0, sizeof(P));
+  P.dev = D;
+  const uint64_t n = D.n, H = D.H, B = D.B, rowb = 128;
+  int nmaps = 0, nseg = 0, start = 0;
+  std::map<std::pair<int, int>, int> rmap;
+  for (int h0 = 0; h0 < D.H;) {
+    int h1 = h0 + 1;
+    while (h1 < D.H && D.dil[h1] == D.dil[h0]) h1++;
+    const int d = D.dil[h0];
+    for (int rho = 0; rho < d; rho++) {
+      const int cnt = lf_sub_len(D.n, d, rho);
+      const int nqb = (cnt + LF_BQ - 1) / LF_BQ;
+      if (nqb == 0) continue;
+      auto key = std::make_pair(d, rho);
+      if (!rmap.count(key)) {
+        if (nmaps + 4 > LF_BW_MAX_MAPS - 2) {
+          snprintf(err, errlen, "tensor-core backward: too many distinct dilation residues");
+          return LF_ERR_UNSUPPORTED;
+        }
+        const char *srcs[4] = {(const char *)a.qs, (const char *)a.ks, (const char *)a.vs,
+                               (const char *)a.dO};
+        for (int k = 0; k < 4; k++)
+          if (!lf_make_map(&P.maps[nmaps + k], f16, srcs[k] + rho * rowb, cnt, H, B, d * rowb,
+                           n * rowb, H * n * rowb, LF_BQ)) {
+            snprintf(err, errlen, "tensor map encode failed (backward, d=%d, rho=%d)", d, rho);
+            return LF_ERR_CUDA;
+          }
+        rmap[key] = nmaps;
+        nmaps += 4;
+      }
+      if (nseg >= LF_BW_MAX_SEG) {
+        snprintf(err, errlen, "tensor-core backward: too many head/residue segments");
+        return LF_ERR_UNSUPPORTED;
+      }
+      P.seg[nseg] = LfTcSeg{h0, h1, d, rho, cnt, nqb, start, rmap[key]};
+      start += (h1 - h0) * nqb;
+      nseg++;
+    }
+    h0 = h1;
+  }
+  P.nseg = nseg;
+  P.per_batch = start;
+  const int Ga = L.ws.G, Gka = L.ws.Gk;
+  char *qg_c = L.ws_base + L.ws.qg_c, *ks_c = L.ws_base + L.ws.ks_c, *vs_c = L.ws_base + L.ws.vs_c;
+  P.gbox = std::min(Gka, LF_BK);
+  P.map_ksc = nmaps;
+  P.map_vsc = nmaps + 1;
+  if (!lf_make_map(&P.maps[nmaps], f16, ks_c, Gka, H, B, rowb, Gka * rowb, H * Gka * rowb, P.gbox) ||
+      !lf_make_map(&P.maps[nmaps + 1], f16, vs_c, Gka, H, B, rowb, Gka * rowb, H * Gka * rowb, P.gbox)) {
+    snprintf(err, errlen, "tensor map encode failed (backward global maps)");
+    return LF_ERR_CUDA;
+  }
+  P.lse = a.lse;
+  P.delta = delta;
+  if (D.G > 0) {
+    ce = lf_launch_gather(L, a.qg, a.ks, a.vs, qg_c, ks_c, vs_c, Ga, Gka);
+    if (ce != cudaSuccess) {
+      snprintf(err, errlen, "gather launch: %s", cudaGetErrorString(ce));
+      return LF_ERR_CUDA;
+    }
+  }
+  static bool attr_done[2][2] = {{false, false}, {false, false}};
+  const unsigned grid = (unsigned)((long long)D.B * P.per_batch);
+  for (int mode = 0; mode < 2; mode++) {  // 0: dK/dV (rows = keys), 1: dQ (rows = queries)
+    void (*kern)(const LfBwParams) =
+        f16 ? (mode ? lf_tc_bwd_kernel<1, 1> : lf_tc_bwd_kernel<1, 0>)
+            : (mode ? lf_tc_bwd_kernel<0, 1> : lf_tc_bwd_kernel<0, 0>);
+    if (!attr_done[f16][mode]) {
+      ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LF_BW_SMEM);
+      if (ce != cudaSuccess) {
+        snprintf(err, errlen, "cudaFuncSetAttribute (backward): %s", cudaGetErrorString(ce));
+        return LF_ERR_CUDA;
+      }
+      attr_done[f16][mode] = true;
+    }
+    P.out0 = mode ? a.dqs : a.dvs;
+    P.out1 = mode ? nullptr : a.dks;
+    kern<<<grid, LF_BW_THREADS, LF_BW_SMEM, L.stream>>>(P);
+    lf_launches_add(1);
+    ce = cudaGetLastError();
+    if (ce != cudaSuccess) {
+      snprintf(err, errlen, "tensor-core backward launch: %s", cudaGetErrorString(ce));
+      return LF_ERR_CUDA;
+    }
+  }
+  // global-column part of dK_s / dV_s (after the band part) and dQ_g
+  const int nch = (D.n + LF_BW_ROWS_PER_CHUNK - 1) / LF_BW_ROWS_PER_CHUNK;
+  float *part_kv = (float *)(L.ws_base + L.ws.part_acc), *part_q = (float *)(L.ws_base + L.ws.part_ml);
+  ce = f16 ? lf_bwd_global_parts<__half>(L, a, delta, part_kv, part_q, nch)
+           : lf_bwd_global_parts<__nv_bfloat16>(L, a, delta, part_kv, part_q, nch);
+  if (ce != cudaSuccess) {
+    snprintf(err, errlen, "backward global parts: %s", cudaGetErrorString(ce));
+    return LF_ERR_CUDA;
+  }
+  return LF_OK;
+}

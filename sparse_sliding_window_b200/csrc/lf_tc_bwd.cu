@@ -421,31 +421,32 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
     // ---- epilogue: accumulators -> gradient rows
     if (alive && lf_wait_warp(o_full, 0, abort_flag, D.status, 30)) {
       lf_tc_fence_after();
-      if (trow < it.cnt) {
-        const size_t orow = bh * n + pos;
+      // TMEM loads are warp-collective: every lane loads, only rows that exist store
+      const bool store = trow < it.cnt;
+      const size_t orow = bh * n + pos;
+      const float keep = active ? 1.f : 0.f;
 #pragma unroll
-        for (int which = 0; which < (kModeQ ? 1 : 2); which++) {
-          float a[32], c2[32];
-          lf_tmem_ld32(tmem + lane_off + (which ? LF_BT_ACC1 : LF_BT_ACC0), a);
-          lf_tmem_ld32(tmem + lane_off + (which ? LF_BT_ACC1 : LF_BT_ACC0) + 32, c2);
-          const float keep = active ? 1.f : 0.f;
-          void *outp = which ? P.out1 : P.out0;
-          uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(outp) + orow * LF_HD);
+      for (int which = 0; which < (kModeQ ? 1 : 2); which++) {
+        float a[32], c2[32];
+        lf_tmem_ld32(tmem + lane_off + (which ? LF_BT_ACC1 : LF_BT_ACC0), a);
+        lf_tmem_ld32(tmem + lane_off + (which ? LF_BT_ACC1 : LF_BT_ACC0) + 32, c2);
+        if (!store) continue;
+        void *outp = which ? P.out1 : P.out0;
+        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(outp) + orow * LF_HD);
 #pragma unroll
-          for (int k = 0; k < 4; k++) {
-            uint4 u;
-            u.x = lf_pack2<kF16>(a[8 * k + 0] * keep, a[8 * k + 1] * keep);
-            u.y = lf_pack2<kF16>(a[8 * k + 2] * keep, a[8 * k + 3] * keep);
-            u.z = lf_pack2<kF16>(a[8 * k + 4] * keep, a[8 * k + 5] * keep);
-            u.w = lf_pack2<kF16>(a[8 * k + 6] * keep, a[8 * k + 7] * keep);
-            dst[k] = u;
-            uint4 v;
-            v.x = lf_pack2<kF16>(c2[8 * k + 0] * keep, c2[8 * k + 1] * keep);
-            v.y = lf_pack2<kF16>(c2[8 * k + 2] * keep, c2[8 * k + 3] * keep);
-            v.z = lf_pack2<kF16>(c2[8 * k + 4] * keep, c2[8 * k + 5] * keep);
-            v.w = lf_pack2<kF16>(c2[8 * k + 6] * keep, c2[8 * k + 7] * keep);
-            dst[4 + k] = v;
-          }
+        for (int k = 0; k < 4; k++) {
+          uint4 u;
+          u.x = lf_pack2<kF16>(a[8 * k + 0] * keep, a[8 * k + 1] * keep);
+          u.y = lf_pack2<kF16>(a[8 * k + 2] * keep, a[8 * k + 3] * keep);
+          u.z = lf_pack2<kF16>(a[8 * k + 4] * keep, a[8 * k + 5] * keep);
+          u.w = lf_pack2<kF16>(a[8 * k + 6] * keep, a[8 * k + 7] * keep);
+          dst[k] = u;
+          uint4 v;
+          v.x = lf_pack2<kF16>(c2[8 * k + 0] * keep, c2[8 * k + 1] * keep);
+          v.y = lf_pack2<kF16>(c2[8 * k + 2] * keep, c2[8 * k + 3] * keep);
+          v.z = lf_pack2<kF16>(c2[8 * k + 4] * keep, c2[8 * k + 5] * keep);
+          v.w = lf_pack2<kF16>(c2[8 * k + 6] * keep, c2[8 * k + 7] * keep);
+          dst[4 + k] = v;
         }
       }
     }

@@ -219,7 +219,9 @@ def time_backward(att, d, wl, pairs, world, args, dev, stream):
         t = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
-    return {"ms_per_step": ms, "steps": k, "kernels": "CUDA-core backward (delta, dQ, dK_s/dV_s, dK_g/dV_g)",
+    kinds = ("CUDA-core backward (delta, dQ, dK_s/dV_s, dK_g/dV_g)" if wl.dtype == "f32" else
+             "tensor-core dQ and dK/dV band kernels + CUDA-core global-token parts")
+    return {"ms_per_step": ms, "steps": k, "kernels": kinds,
             "tflops_algorithmic": 8.0 * wl.head_dim * pairs * world / (ms * 1e-3) / 1e12,
             "scores_per_s": pairs * world / (ms * 1e-3)}
 

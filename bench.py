@@ -117,6 +117,41 @@ class ClockSampler:
                 "samples": len(sm), "window": "warm-up and timed region"}
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest of the per-rank values (device timings are reported as the
+    slowest rank).  Uses the default process group when world > 1."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job units per second: every rank processes its own replica of
+    the workload (weak scaling); the step time is the slowest rank's."""
+    return units_per_rank * world / (ms_per_step * 1e-3)
+
+
+# DRAM traffic of the main forward kernel per launch, from the ncu captures
+# summarised under profiles/; reported only while the kernel sources are the
+# ones that were profiled (their sha256 prefix), else null.
+PROFILED_TRAFFIC = {"base_bf16": {"bytes": 31915776, "sha": "2475438af35076a3"}}
+
+
+def kernel_traffic(workload: str):
+    import hashlib
+    rec = PROFILED_TRAFFIC.get(workload)
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for f in ("lf_tc.cu", "lf_ptx.cuh", "lf_common.cuh"):
+        h.update(open(os.path.join(ROOT, "sparse_sliding_window_b200", "csrc", f), "rb").read())
+    return rec["bytes"] if h.hexdigest()[:16] == rec["sha"] else None
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -214,11 +249,7 @@ def time_backward(att, d, wl, pairs, world, args, dev, stream):
         bstep()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1) / k
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / k, world, dev)
     kinds = ("CUDA-core backward (delta, dQ, dK_s/dV_s, dK_g/dV_g)" if wl.dtype == "f32" else
              "tensor-core dQ and dK/dV band kernels + CUDA-core global-token parts")
     return {"ms_per_step": ms, "steps": k, "kernels": kinds,
@@ -334,10 +365,7 @@ def main():
     t_ms = e0.elapsed_time(e1)
     k_ms = float(np.mean([a.elapsed_time(b) for a, b in kev]))
     att.status()
-    if world > 1:
-        t = torch.tensor([t_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_ms = float(t.item())
+    t_ms = max_over_ranks(t_ms, world, dev)
     ms_step_eager = t_ms / args.steps
     ms_step = ms_step_eager
     if not args.no_graph:
@@ -366,15 +394,11 @@ def main():
             graphs[k % nsets].replay()
         g1.record(stream)
         torch.cuda.synchronize(dev)
-        gt_ms = g0.elapsed_time(g1)
-        if world > 1:
-            t = torch.tensor([gt_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            gt_ms = float(t.item())
+        gt_ms = max_over_ranks(g0.elapsed_time(g1), world, dev)
         ms_step = gt_ms / args.steps
         att.status()
         del graphs
-    value = pairs * world / (ms_step * 1e-3)
+    value = job_throughput(pairs, world, ms_step)
     flops = 4.0 * wl.head_dim * pairs
     tflops = flops * world / (ms_step * 1e-3) / 1e12
 
@@ -398,11 +422,7 @@ def main():
         o_host.copy_(d["o"], non_blocking=True)
     ee1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = ee0.elapsed_time(ee1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(ee0.elapsed_time(ee1) / e2e_steps, world, dev)
     h2d = set_bytes + host["mask"].numel() * 4
     d2h = o_host.numel() * o_host.element_size()
 
@@ -416,7 +436,7 @@ def main():
     else:
         roof = {"bound": "tensor", "achieved": flops / k_s / 1e12, "peak": pk["bf16"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = kernel_traffic(wl.name) if args.kernel != "simt" else None
     roof["peak_source"] = pk["src"]
     roof["kernel_ms"] = k_ms
     roof["algorithmic_bytes"] = abytes

@@ -171,25 +171,89 @@ cudaError_t lf_launch_dump(const LfLaunch &L, uint8_t *out) {
 
 // ========================================================= CUDA-core fwd
 
-struct LfRowState {
-  float mx, l, a0, a1;
-};
-
-// Online softmax step for key row koff (element offset of lane's pair).
+// 64 elements of a row as float
 template <typename T>
-__device__ __forceinline__ void lf_visit(LfRowState &st, float2 q, const T *K, const T *V,
-                                         size_t koff) {
-  float2 k = LfIo<T>::ld2(K + koff);
-  float s = lf_warp_sum(q.x * k.x + q.y * k.y);  // log2 domain (q pre-scaled)
-  float mn = fmaxf(st.mx, s);
-  float al = exp2f(st.mx - mn);
-  float pr = exp2f(s - mn);
-  float2 v = LfIo<T>::ld2(V + koff);
-  st.l = st.l * al + pr;
-  st.a0 = st.a0 * al + pr * v.x;
-  st.a1 = st.a1 * al + pr * v.y;
-  st.mx = mn;
+__device__ __forceinline__ void lf_load_row64(const T *p, float (&x)[64]);
+template <>
+__device__ __forceinline__ void lf_load_row64<float>(const float *p, float (&x)[64]) {
+  const float4 *q = reinterpret_cast<const float4 *>(p);
+#pragma unroll
+  for (int k = 0; k < 16; k++) {
+    const float4 v = q[k];
+    x[4 * k] = v.x;
+    x[4 * k + 1] = v.y;
+    x[4 * k + 2] = v.z;
+    x[4 * k + 3] = v.w;
+  }
 }
+template <typename H2, typename T>
+__device__ __forceinline__ void lf_load_row64_h(const T *p, float (&x)[64]) {
+  const uint4 *q = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+  for (int k = 0; k < 8; k++) {
+    const uint4 v = q[k];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const float2 f = LfIo<T>::ld2(reinterpret_cast<const T *>(&w[j]));
+      x[8 * k + 2 * j] = f.x;
+      x[8 * k + 2 * j + 1] = f.y;
+    }
+  }
+}
+template <>
+__device__ __forceinline__ void lf_load_row64<__nv_bfloat16>(const __nv_bfloat16 *p, float (&x)[64]) {
+  lf_load_row64_h<__nv_bfloat162>(p, x);
+}
+template <>
+__device__ __forceinline__ void lf_load_row64<__half>(const __half *p, float (&x)[64]) {
+  lf_load_row64_h<__half2>(p, x);
+}
+
+// One warp per query row, keys in batches of 32 (one key per lane): the lane
+// forms its key's full score, the warp updates the running max / sum, then
+// every lane accumulates its two output columns over the batch's keys.
+template <typename T>
+struct LfRowAcc {
+  float q[64];
+  float mx, l, a0, a1;
+  __device__ __forceinline__ void batch(const T *K, const T *V, size_t base, int j, bool ok, int lane) {
+    float s = -INFINITY;
+    if (ok) {
+      float k[64];
+      lf_load_row64<T>(K + base + (size_t)j * LF_HD, k);
+      float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; c += 4) {
+        d0 = fmaf(q[c], k[c], d0);
+        d1 = fmaf(q[c + 1], k[c + 1], d1);
+        d2 = fmaf(q[c + 2], k[c + 2], d2);
+        d3 = fmaf(q[c + 3], k[c + 3], d3);
+      }
+      s = (d0 + d1) + (d2 + d3);  // q is pre-scaled by scale * log2(e)
+    }
+    float bm = s;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+    if (bm == -INFINITY) return;  // no key in this batch (warp-uniform)
+    const float mn = fmaxf(mx, bm);
+    const float al = exp2f(mx - mn);
+    const float p = ok ? exp2f(s - mn) : 0.f;
+    l = l * al + lf_warp_sum(p);
+    a0 *= al;
+    a1 *= al;
+    const unsigned live = __ballot_sync(0xffffffffu, ok);
+    for (unsigned bits = live; bits; bits &= bits - 1) {
+      const int src = __ffs(bits) - 1;
+      const float pj = __shfl_sync(0xffffffffu, p, src);
+      const int jj = __shfl_sync(0xffffffffu, j, src);
+      const float2 v = LfIo<T>::ld2(V + base + (size_t)jj * LF_HD + 2 * lane);
+      a0 = fmaf(pj, v.x, a0);
+      a1 = fmaf(pj, v.y, a1);
+    }
+    mx = mn;
+  }
+};
 
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -202,8 +266,8 @@ __global__ void __launch_bounds__(256)
   const int i = (int)(row % n);
   const int bh = (int)(row / n), h = bh % P.H, b = bh / P.H, d = P.dil[h];
   const int32_t *m = P.mask + (size_t)b * n;
-  const size_t base = (size_t)bh * n * LF_HD + 2 * lane;
-  const size_t ooff = base + (size_t)i * LF_HD;
+  const size_t base = (size_t)bh * n * LF_HD;
+  const size_t ooff = base + (size_t)i * LF_HD + 2 * lane;
   const int code = m[i];
   if (code == 0) {
     LfIo<T>::st2(o + ooff, 0.f, 0.f);
@@ -212,25 +276,30 @@ __global__ void __launch_bounds__(256)
   }
   const bool glob = code == 2;
   const T *Q = glob ? qg : qs, *K = glob ? kg : ks, *V = glob ? vg : vs;
-  float2 q = LfIo<T>::ld2(Q + ooff);
-  q.x *= P.scale_log2;
-  q.y *= P.scale_log2;
-  LfRowState st{-INFINITY, 0.f, 0.f, 0.f};
+  LfRowAcc<T> st;
+  lf_load_row64<T>(Q + base + (size_t)i * LF_HD, st.q);
+#pragma unroll
+  for (int c = 0; c < 64; c++) st.q[c] *= P.scale_log2;
+  st.mx = -INFINITY;
+  st.l = st.a0 = st.a1 = 0.f;
   if (glob) {
-    for (int j = 0; j < n; j++)
-      if (m[j] != 0) lf_visit<T>(st, q, K, V, base + (size_t)j * LF_HD);
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
+      st.batch(K, V, base, j, j < n && m[j] != 0, lane);
+    }
   } else {
+    // window keys j = i + k*d, k in [-r, khi], then the global keys outside it
     const int khi = P.causal ? 0 : P.r;
-    for (int k = -P.r; k <= khi; k++) {
-      int j = i + k * d;
-      if (j < 0 || j >= n || m[j] == 0) continue;
-      lf_visit<T>(st, q, K, V, base + (size_t)j * LF_HD);
+    for (int k0 = -P.r; k0 <= khi; k0 += 32) {
+      const int k = k0 + lane, j = i + k * d;
+      st.batch(K, V, base, j, k <= khi && j >= 0 && j < n && m[j] != 0, lane);
     }
     const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
     const int32_t *gl = P.gidx + (size_t)b * P.G;
-    for (int t = 0; t < ng; t++) {
-      int g = gl[t];
-      if (!lf_in_window(i, g, P.r, d, P.causal)) lf_visit<T>(st, q, K, V, base + (size_t)g * LF_HD);
+    for (int t0 = 0; t0 < ng; t0 += 32) {
+      const int t = t0 + lane;
+      const int g = t < ng ? gl[t] : 0;
+      st.batch(K, V, base, g, t < ng && !lf_in_window(i, g, P.r, d, P.causal), lane);
     }
   }
   const float inv = 1.f / st.l;

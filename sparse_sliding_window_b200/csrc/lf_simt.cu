@@ -217,6 +217,7 @@ template <typename T>
 struct LfRowAcc {
   float q[64];
   float mx, l, a0, a1;
+  int self;  // this warp's own row (a valid address for lanes without a key)
   __device__ __forceinline__ void batch(const T *K, const T *V, size_t base, int j, bool ok, int lane) {
     float s = -INFINITY;
     if (ok) {
@@ -242,21 +243,27 @@ struct LfRowAcc {
     l = l * al + lf_warp_sum(p);
     a0 *= al;
     a1 *= al;
-    const unsigned live = __ballot_sync(0xffffffffu, ok);
-    for (unsigned bits = live; bits; bits &= bits - 1) {
-      const int src = __ffs(bits) - 1;
+    // all 32 value rows of the batch are loaded before the sums (one
+    // latency per batch); a lane without a key points at row `self` with p = 0
+    const int js = ok ? j : self;
+    float2 v[32];
+#pragma unroll
+    for (int src = 0; src < 32; src++) {
+      const int jj = __shfl_sync(0xffffffffu, js, src);
+      v[src] = LfIo<T>::ld2(V + base + (size_t)jj * LF_HD + 2 * lane);
+    }
+#pragma unroll
+    for (int src = 0; src < 32; src++) {
       const float pj = __shfl_sync(0xffffffffu, p, src);
-      const int jj = __shfl_sync(0xffffffffu, j, src);
-      const float2 v = LfIo<T>::ld2(V + base + (size_t)jj * LF_HD + 2 * lane);
-      a0 = fmaf(pj, v.x, a0);
-      a1 = fmaf(pj, v.y, a1);
+      a0 = fmaf(pj, v[src].x, a0);
+      a1 = fmaf(pj, v[src].y, a1);
     }
     mx = mn;
   }
 };
 
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 1)
     lf_simt_fwd_kernel(LfDev P, const T *qs, const T *ks, const T *vs, const T *qg, const T *kg,
                        const T *vg, T *o, float *lse) {
   const int lane = threadIdx.x & 31;
@@ -282,6 +289,7 @@ __global__ void __launch_bounds__(256)
   for (int c = 0; c < 64; c++) st.q[c] *= P.scale_log2;
   st.mx = -INFINITY;
   st.l = st.a0 = st.a1 = 0.f;
+  st.self = i;
   if (glob) {
     for (int j0 = 0; j0 < n; j0 += 32) {
       const int j = j0 + lane;

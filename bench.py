@@ -257,6 +257,55 @@ def time_backward(att, d, wl, pairs, world, args, dev, stream):
             "scores_per_s": pairs * world / (ms * 1e-3)}
 
 
+def run_decode(args, wl):
+    """Decode step of a causal workload: one new token per sequence against
+    the full-length cache (every head), timed on the device.  HBM-bound:
+    the window's key and value rows are read once per head."""
+    import torch
+    from sparse_sliding_window_b200 import lf_attn as L
+    assert wl.causal, "the decode step is the causal window"
+    dev = torch.device("cuda", 0)
+    inp = synth.make_inputs(wl, with_do=False)
+    tdt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[wl.dtype]
+
+    def dev_t(a):
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if wl.dtype == "bf16" else torch.from_numpy(a)
+        return t.to(dev)
+    kc, vc = dev_t(inp["ks"]), dev_t(inp["vs"])
+    q = dev_t(np.ascontiguousarray(inp["qs"][:, :, -1]))
+    lens = torch.full((wl.B,), wl.n, dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((wl.B, wl.H), dtype=torch.float32, device=dev)
+    p = L.make_params(wl.B, wl.H, wl.n, wl.r, wl.dilation, True, 0.0,
+                      {"bf16": L.LF_BF16, "f16": L.LF_F16, "f32": L.LF_F32}[wl.dtype])
+    for _ in range(max(3, args.warmup)):
+        L.lf_attn_decode(p, q, kc, vc, lens, o, lse)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        L.lf_attn_decode(p, q, kc, vc, lens, o, lse)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    eb = 4 if wl.dtype == "f32" else 2
+    keys = sum(min(wl.r, (wl.n - 1) // d) + 1 for d in wl.dilation) * wl.B
+    nbytes = keys * 2 * 64 * eb + 2 * wl.B * wl.H * 64 * eb + wl.B * wl.H * 4
+    pk = _peaks()
+    line = {"metric": "decode tokens/s (causal window, one new token per sequence, all heads)",
+            "value": wl.B / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": wl.dtype,
+            "data": "synthetic", "config": {"workload": wl.name + " decode", "B": wl.B, "H": wl.H,
+                                            "cache_len": wl.n, "window_one_sided": wl.r,
+                                            "dilation": wl.dilation},
+            "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": pk["hbm"],
+                         "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm"],
+                         "traffic": None, "algorithmic_bytes": nbytes,
+                         "note": "timed per launch, so the figure includes launch overhead"}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -269,6 +318,8 @@ def main():
     ap.add_argument("--min-warm-seconds", type=float, default=1.0)
     ap.add_argument("--no-graph", action="store_true",
                     help="time eager launches only (default: also replay each step from a CUDA graph)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the causal-window decode step instead (causal workloads)")
     ap.add_argument("--bwd", action="store_true",
                     help="also time the backward (default for workloads with a backward)")
     args = ap.parse_args()
@@ -279,6 +330,8 @@ def main():
     import torch
     from sparse_sliding_window_b200 import lf_attn as L
 
+    if args.decode:
+        return run_decode(args, wl)
     world, rank, local = _dist()
     if world > 1:
         import datetime

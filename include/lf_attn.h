@@ -115,6 +115,24 @@ int lf_attn_bwd(const lf_attn_params *p, const void *q_s, const void *k_s,
                 void *dv_s, void *dq_g, void *dk_g, void *dv_g,
                 void *workspace, size_t ws_bytes, void *stream);
 
+/* Decode step of the causal (autoregressive) window: one new query per
+ * sequence against a key/value cache ("Longformer：处理长文档的Transformer模型",
+ * segmentfault, 实现: autoregressive language modelling with dilated
+ * sliding windows).  p->causal must be 1; window r and per-head dilation d
+ * as for the forward; there are no global tokens.  For sequence b with
+ * lengths[b] = L >= 1 valid cache rows (the new token's own key and value
+ * already appended at row L-1), the query q[b,h] attends the keys
+ * j = (L-1) - k*d, k = 0..r, j >= 0.
+ *   q        [B,H,64]     the new tokens' queries (device)
+ *   k_cache, v_cache  [B,H,n,64]  cached keys / values, rows >= L unused
+ *   lengths  int32 [B]    device
+ *   o        [B,H,64]     output (overwritten); lse float32 [B,H] or NULL
+ * Returns LF_ERR_INVALID for bad arguments; a length outside [1, n] gives
+ * o = 0 and lse = -inf for that sequence.  Allocates nothing. */
+int lf_attn_decode(const lf_attn_params *p, const void *q, const void *k_cache,
+                   const void *v_cache, const int32_t *lengths, void *o,
+                   float *lse, void *stream);
+
 /* Attended (query, key) pairs per (b, h) -> counts int64 [B, H] (device),
  * enumerated with the tile walk and predicates of the forward kernels.
  * workspace: >= lf_attn_workspace_size(p, 0). */

@@ -125,7 +125,7 @@ static int lf_prepare(const lf_attn_params *p, int for_bwd, LfDev &dev, LfWs &ws
       off = lf_align(off + B * H * Ga * dev.nch * 8);
     } else {
       // backward: per-chunk partials of the global columns (dK, dV) and rows (dQ_g)
-      const size_t nchb = ((size_t)n + 255) / 256;
+      const size_t nchb = ((size_t)n + 63) / 64;  // rows per chunk of the global parts
       ws.part_acc = off;
       off = lf_align(off + B * H * Ga * nchb * 2 * LF_HD * 4);
       ws.part_ml = off;
@@ -238,6 +238,25 @@ extern "C" int lf_attn_bwd(const lf_attn_params *p, const void *q_s, const void 
   return lf_cuda(lf_launch_simt_bwd(L, q_s, k_s, v_s, q_g, k_g, v_g, o, lse, d_o, dq_s, dk_s, dv_s,
                                     dq_g, dk_g, dv_g),
                  "backward");
+}
+
+extern "C" int lf_attn_decode(const lf_attn_params *p, const void *q, const void *k_cache,
+                              const void *v_cache, const int32_t *lengths, void *o, float *lse,
+                              void *stream) {
+  int st;
+  if ((st = lf_check_ptr(q, "q")) || (st = lf_check_ptr(k_cache, "k_cache")) ||
+      (st = lf_check_ptr(v_cache, "v_cache")) || (st = lf_check_ptr(lengths, "lengths")) ||
+      (st = lf_check_ptr(o, "o")) || (st = lf_check_ptr(lse, "lse", true)))
+    return st;
+  LfLaunch L;
+  LfWs ws;
+  if ((st = lf_prepare(p, 0, L.dev, ws))) return st;
+  if (!p->causal) return lf_fail(LF_ERR_INVALID, "the decode step is the causal window: set causal = 1");
+  L.ws = ws;
+  L.ws_base = nullptr;
+  L.stream = (cudaStream_t)stream;
+  L.dtype = p->dtype;
+  return lf_cuda(lf_launch_decode(L, q, k_cache, v_cache, lengths, o, lse), "decode");
 }
 
 extern "C" int lf_attn_count_pairs(const lf_attn_params *p, const int32_t *mask, int64_t *counts,

@@ -165,6 +165,8 @@ struct LfLaunch {
 
 cudaError_t lf_launch_mask_pass(const LfLaunch &L);
 cudaError_t lf_launch_count(const LfLaunch &L, int64_t *counts);
+cudaError_t lf_launch_decode(const LfLaunch &L, const void *q, const void *kc, const void *vc,
+                             const int32_t *lengths, void *o, float *lse);
 cudaError_t lf_launch_dump(const LfLaunch &L, uint8_t *out);
 cudaError_t lf_launch_simt_fwd(const LfLaunch &L, const void *qs, const void *ks, const void *vs,
                                const void *qg, const void *kg, const void *vg, void *o, float *lse);

@@ -556,3 +556,84 @@ cudaError_t lf_launch_bwd_delta_dkvg(const LfLaunch &L, const void *o, const voi
     return lf_bwd_delta_dkvg_t<__nv_bfloat16>(L, o, dO, delta, qg, kg, vg, lse, dkg, dvg);
   return lf_bwd_delta_dkvg_t<float>(L, o, dO, delta, qg, kg, vg, lse, dkg, dvg);
 }
+
+// ============================================================ decode step
+
+// One block of 8 warps per (b, h): warp w takes the window offsets
+// k = w*32*chunks ... (one key per lane, batches of 32), then the warps merge
+// their (max, sum, partial output) in shared memory.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    lf_decode_kernel(LfDev P, const T *q, const T *kc, const T *vc, const int32_t *lengths, T *o,
+                     float *lse) {
+  __shared__ float s_m[8], s_l[8], s_acc[8][LF_HD];
+  const int bh = blockIdx.x, h = bh % P.H, b = bh / P.H, d = P.dil[h], n = P.n;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int L = lengths[b];
+  const size_t obase = (size_t)bh * LF_HD;
+  if (L < 1 || L > n) {
+    if (warp == 0) {
+      LfIo<T>::st2(o + obase + 2 * lane, 0.f, 0.f);
+      if (lse && lane == 0) lse[bh] = -INFINITY;
+    }
+    return;
+  }
+  const int t = L - 1;
+  const int kmax = min(P.r, t / d);  // keys j = t - k*d >= 0
+  const size_t base = (size_t)bh * n * LF_HD;
+  LfRowAcc<T> st;
+  lf_load_row64<T>(q + obase, st.q);
+#pragma unroll
+  for (int c = 0; c < 64; c++) st.q[c] *= P.scale_log2;
+  st.mx = -INFINITY;
+  st.l = st.a0 = st.a1 = 0.f;
+  st.self = t;
+  for (int k0 = warp * 32; k0 <= kmax; k0 += 8 * 32) {
+    const int k = k0 + lane;
+    st.batch(kc, vc, base, t - k * d, k <= kmax, lane);
+  }
+  if (lane == 0) {
+    s_m[warp] = st.mx;
+    s_l[warp] = st.l;
+  }
+  s_acc[warp][2 * lane] = st.a0;
+  s_acc[warp][2 * lane + 1] = st.a1;
+  __syncthreads();
+  if (warp == 0) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 8; w++) M = fmaxf(M, s_m[w]);
+    float Ls = 0.f, a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; w++) {
+      if (s_m[w] == -INFINITY) continue;
+      const float f = exp2f(s_m[w] - M);
+      Ls += s_l[w] * f;
+      a0 += s_acc[w][2 * lane] * f;
+      a1 += s_acc[w][2 * lane + 1] * f;
+    }
+    LfIo<T>::st2(o + obase + 2 * lane, a0 / Ls, a1 / Ls);
+    if (lse && lane == 0) lse[bh] = (M + log2f(Ls)) * LF_LN2;
+  }
+}
+
+cudaError_t lf_launch_decode(const LfLaunch &L, const void *q, const void *kc, const void *vc,
+                             const int32_t *lengths, void *o, float *lse) {
+  const unsigned grid = (unsigned)(L.dev.B * L.dev.H);
+  switch (L.dtype) {
+    case LF_F32:
+      lf_decode_kernel<float><<<grid, 256, 0, L.stream>>>(L.dev, (const float *)q, (const float *)kc,
+                                                          (const float *)vc, lengths, (float *)o, lse);
+      break;
+    case LF_BF16:
+      lf_decode_kernel<__nv_bfloat16><<<grid, 256, 0, L.stream>>>(
+          L.dev, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)kc, (const __nv_bfloat16 *)vc,
+          lengths, (__nv_bfloat16 *)o, lse);
+      break;
+    default:
+      lf_decode_kernel<__half><<<grid, 256, 0, L.stream>>>(L.dev, (const __half *)q, (const __half *)kc,
+                                                           (const __half *)vc, lengths, (__half *)o, lse);
+  }
+  lf_launches_add(1);
+  return cudaGetLastError();
+}

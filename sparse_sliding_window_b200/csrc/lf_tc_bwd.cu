@@ -43,7 +43,7 @@
 #define LF_BW_NS 3
 #define LF_BW_MAX_MAPS 40
 #define LF_BW_MAX_SEG 32
-#define LF_BW_ROWS_PER_CHUNK 256  // rows (keys) per warp of the global-row / -column parts
+#define LF_BW_ROWS_PER_CHUNK 64  // rows (keys) per warp of the global-row / -column parts
 
 #define LF_BW_R0 0
 #define LF_BW_R1 16384

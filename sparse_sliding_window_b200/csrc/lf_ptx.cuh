@@ -126,6 +126,112 @@ __device__ __forceinline__ void lf_mma_ts(uint32_t d, uint32_t a, uint64_t b, ui
       : "memory");
 }
 
+// ---- MMA phases issued by a converged warp.  One elected lane (the same
+// lane every time the full warp is converged) issues a whole phase from a
+// single asm statement.  Issue cost measured on B200: one tcgen05.mma per
+// asm statement from a diverged lane ~180 cycles each; a four-MMA S phase
+// (128x128x64) as one statement ~380 cycles, an eight-MMA P.V phase
+// (128x64x128) ~490 -- against 256 + 256 cycles of tensor-core work.  Every
+// tcgen05 operation of the warp comes from that lane, so each commit tracks
+// all of them.
+
+// commit of all prior MMAs of the warp to `bar`
+__device__ __forceinline__ void lf_commit_w(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          bar)
+      : "memory");
+}
+
+// D = A * B^T over a 64-wide reduction: four K = 16 MMAs with K-major
+// 128-byte-swizzled operands (each descriptor advances 32 bytes per step,
+// i.e. +2 in its 16-byte units), then a commit to `bar`.
+__device__ __forceinline__ void lf_mma_s_phase(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                               uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+      "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+      "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, 1;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%4];\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(bar)
+      : "memory");
+}
+
+// Two such products into two accumulators (D0 = A0 B0^T, D1 = A1 B1^T,
+// same shape), interleaved step by step, then one commit to `bar`.
+__device__ __forceinline__ void lf_mma_s2_phase(uint32_t d0, uint64_t a0, uint64_t b0, uint32_t d1,
+                                                uint64_t a1, uint64_t b1, uint32_t idesc,
+                                                uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b64 x1, x2, x3, y1, y2, y3, u1, u2, u3, v1, v2, v3;\n\t"
+      "add.s64 x1, %1, 2;\n\tadd.s64 x2, %1, 4;\n\tadd.s64 x3, %1, 6;\n\t"
+      "add.s64 y1, %2, 2;\n\tadd.s64 y2, %2, 4;\n\tadd.s64 y3, %2, 6;\n\t"
+      "add.s64 u1, %4, 2;\n\tadd.s64 u2, %4, 4;\n\tadd.s64 u3, %4, 6;\n\t"
+      "add.s64 v1, %5, 2;\n\tadd.s64 v2, %5, 4;\n\tadd.s64 v3, %5, 6;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %6, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%3], %4, %5, %6, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], x1, y1, %6, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%3], u1, v1, %6, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], x2, y2, %6, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%3], u2, v2, %6, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], x3, y3, %6, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%3], u3, v3, %6, 1;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t}" ::"r"(d0),
+      "l"(a0), "l"(b0), "r"(d1), "l"(a1), "l"(b1), "r"(idesc), "r"(bar)
+      : "memory");
+}
+
+// D (+)= A * B with A in TMEM: up to eight K = 16 MMAs, step k reading A
+// columns a + 8k and the B descriptor advanced by bstep * k (16-byte units);
+// step k is issued when bit k of kmask is set (kmask = 2^steps - 1, steps
+// >= 1).  Step 0 accumulates iff acc0 != 0, later steps always do.  Then
+// commits to bar1, bar2 and bar3, each skipped when its address is 0.
+__device__ __forceinline__ void lf_mma_ts_phase(uint32_t d, uint32_t a, uint64_t b, uint32_t bstep,
+                                                uint32_t idesc, uint32_t kmask, uint32_t acc0,
+                                                uint32_t bar1, uint32_t bar2, uint32_t bar3) {
+  asm volatile(
+      "{\n\t.reg .pred e, pa, p1, p2, p3, p4, p5, p6, p7, c1, c2, c3;\n\t"
+      ".reg .b32 t1, t2, t3, t4, t5, t6, t7, m;\n\t.reg .b64 s, b1, b2, b3, b4, b5, b6, b7;\n\t"
+      "add.u32 t1, %1, 8;\n\tadd.u32 t2, %1, 16;\n\tadd.u32 t3, %1, 24;\n\tadd.u32 t4, %1, 32;\n\t"
+      "add.u32 t5, %1, 40;\n\tadd.u32 t6, %1, 48;\n\tadd.u32 t7, %1, 56;\n\t"
+      "cvt.u64.u32 s, %4;\n\t"
+      "add.s64 b1, %2, s;\n\tadd.s64 b2, b1, s;\n\tadd.s64 b3, b2, s;\n\tadd.s64 b4, b3, s;\n\t"
+      "add.s64 b5, b4, s;\n\tadd.s64 b6, b5, s;\n\tadd.s64 b7, b6, s;\n\t"
+      "setp.ne.b32 pa, %6, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "and.b32 m, %5, 2;\n\tsetp.ne.and.b32 p1, m, 0, e;\n\t"
+      "and.b32 m, %5, 4;\n\tsetp.ne.and.b32 p2, m, 0, e;\n\t"
+      "and.b32 m, %5, 8;\n\tsetp.ne.and.b32 p3, m, 0, e;\n\t"
+      "and.b32 m, %5, 16;\n\tsetp.ne.and.b32 p4, m, 0, e;\n\t"
+      "and.b32 m, %5, 32;\n\tsetp.ne.and.b32 p5, m, 0, e;\n\t"
+      "and.b32 m, %5, 64;\n\tsetp.ne.and.b32 p6, m, 0, e;\n\t"
+      "and.b32 m, %5, 128;\n\tsetp.ne.and.b32 p7, m, 0, e;\n\t"
+      "setp.ne.and.b32 c1, %7, 0, e;\n\t"
+      "setp.ne.and.b32 c2, %8, 0, e;\n\t"
+      "setp.ne.and.b32 c3, %9, 0, e;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, pa;\n\t"
+      "@p1 tcgen05.mma.cta_group::1.kind::f16 [%0], [t1], b1, %3, 1;\n\t"
+      "@p2 tcgen05.mma.cta_group::1.kind::f16 [%0], [t2], b2, %3, 1;\n\t"
+      "@p3 tcgen05.mma.cta_group::1.kind::f16 [%0], [t3], b3, %3, 1;\n\t"
+      "@p4 tcgen05.mma.cta_group::1.kind::f16 [%0], [t4], b4, %3, 1;\n\t"
+      "@p5 tcgen05.mma.cta_group::1.kind::f16 [%0], [t5], b5, %3, 1;\n\t"
+      "@p6 tcgen05.mma.cta_group::1.kind::f16 [%0], [t6], b6, %3, 1;\n\t"
+      "@p7 tcgen05.mma.cta_group::1.kind::f16 [%0], [t7], b7, %3, 1;\n\t"
+      "@c1 tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t"
+      "@c2 tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%8];\n\t"
+      "@c3 tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%9];\n\t}" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(bstep), "r"(kmask), "r"(acc0), "r"(bar1), "r"(bar2),
+      "r"(bar3)
+      : "memory");
+}
+
 // 32 consecutive fp32 columns of this thread's TMEM lane
 __device__ __forceinline__ void lf_tmem_ld32(uint32_t taddr, float (&x)[32]) {
   uint32_t r[32];

@@ -335,83 +335,98 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
     }
   } else if (warp == 9) {
     // ================================================== MMA issuer
-    if (lane == 0) {
-      const uint64_t dq0 = lf_sdesc(sbase + LF_SM_Q(0), 16, 1024);
-      const uint64_t dk0 = lf_sdesc(sbase + LF_SM_K(0), 16, 1024);
-      const uint64_t dv0 = lf_sdesc(sbase + LF_SM_V(0), 0, 1024);
-      const uint32_t id_pv = lf_idesc(kF16, 64, 1), id_s = lf_idesc(kF16, LF_BK, 0);
-      int gt = 0, k = 0, pc[2] = {0, 0};
-      bool ok = true;
-      for (int idx = blockIdx.x; idx < nitems && ok; idx += gridDim.x) {
-        LfItem it;
-        if (!lf_decode(P, idx, it)) continue;
-        const int qb = k & 1;
-        const int ngk = (it.ng + 15) / 16 * 16;  // global key tile width, multiple of 16
-        auto ncols = [&](int t) { return t < it.nband ? LF_BK : min(LF_BK, ngk - (t - it.nband) * LF_BK); };
-        auto issue_s = [&](int t) {
-          const int s = (gt + t) % LF_TC_NS, g = t & 1;
-          const uint64_t dq = dq0 + (uint64_t)(qb * (16384 >> 4));
-          const uint64_t dk = dk0 + (uint64_t)(s * (32768 >> 4));
-          const uint32_t id = t < it.nband ? id_s : lf_idesc(kF16, ncols(t), 0);
-#pragma unroll
-          for (int kk = 0; kk < 4; kk++)
-            lf_mma_ss(tmem + LF_TM_S(g), dq + 2 * kk, dk + 2 * kk, id, kk > 0);
-        };
-        if (!lf_wait_fast(q_full0 + 8 * qb, (k >> 1) & 1, abort_flag, D.status, 3)) {
+    // The whole warp walks the tile stream and waits together; one elected
+    // lane issues each MMA phase.  Order per tile t of group g = t & 1:
+    // wait P_g(t), issue the group's next S (tile t + 2, or at the end of
+    // the item the group's first tile of the next item, so the softmax
+    // finds it ready after the merge), then O_g += P_g V_t.
+    const uint64_t dq0 = lf_sdesc(sbase + LF_SM_Q(0), 16, 1024);
+    const uint64_t dk0 = lf_sdesc(sbase + LF_SM_K(0), 16, 1024);
+    const uint64_t dv0 = lf_sdesc(sbase + LF_SM_V(0), 0, 1024);
+    const uint32_t id_pv = lf_idesc(kF16, 64, 1);
+    int gt = 0, k = 0;
+    uint32_t pc = 0;  // bit g: parity of group g's next p_full phase
+    bool ok = true;
+    // S of tile t of item `it` (Q buffer qb, ring position gtt) into S_g
+    auto issue_s = [&](const LfItem &it, int qb, int t, int gtt) -> bool {
+      const int s = gtt % LF_TC_NS;
+      if (!lf_wait_warp(kv_full0 + 8 * s, (gtt / LF_TC_NS) & 1, abort_flag, D.status, 4)) return false;
+      lf_tc_fence_after();
+      const int ngk = (it.ng + 15) / 16 * 16;  // global key tile width, multiple of 16
+      const int nc = t < it.nband ? LF_BK : min(LF_BK, ngk - (t - it.nband) * LF_BK);
+      lf_mma_s_phase(tmem + LF_TM_S(t & 1), dq0 + (uint64_t)(qb * (16384 >> 4)),
+                     dk0 + (uint64_t)(s * (32768 >> 4)), lf_idesc(kF16, nc, 0), s_full(t & 1));
+      return true;
+    };
+    int idx = blockIdx.x;
+    LfItem it;
+    bool have = false;
+    for (; idx < nitems; idx += gridDim.x)
+      if (lf_decode(P, idx, it)) {
+        have = true;
+        break;
+      }
+    uint32_t pre = 0;  // bit t: S of tile t (< 2) of `it` already issued
+    while (have && ok) {
+      const int qb = k & 1;
+      if (!lf_wait_warp(q_full0 + 8 * qb, (k >> 1) & 1, abort_flag, D.status, 3)) {
+        ok = false;
+        break;
+      }
+      for (int t = 0; t < 2 && t < it.T && ok; t++)
+        if (!((pre >> t) & 1u)) ok = issue_s(it, qb, t, gt + t);
+      if (!ok) break;
+      // the next item of this CTA
+      LfItem nx;
+      bool have_nx = false;
+      int nidx = idx + gridDim.x;
+      for (; nidx < nitems; nidx += gridDim.x)
+        if (lf_decode(P, nidx, nx)) {
+          have_nx = true;
+          break;
+        }
+      uint32_t npre = 0;
+      bool nq_ready = false;
+      for (int t = 0; t < it.T && ok; t++) {
+        const int g = t & 1;
+        // P(t) written and S(t) consumed by softmax group g
+        if (!lf_wait_warp(p_full(g), (pc >> g) & 1u, abort_flag, D.status, 5)) {
           ok = false;
           break;
         }
-        for (int t = 0; t < 2 && t < it.T; t++) {
-          const int s = (gt + t) % LF_TC_NS;
-          if (!lf_wait_fast(kv_full0 + 8 * s, ((gt + t) / LF_TC_NS) & 1, abort_flag, D.status, 4)) {
-            ok = false;
-            break;
+        pc ^= 1u << g;
+        lf_tc_fence_after();
+        if (t + 2 < it.T) {
+          ok = issue_s(it, qb, t + 2, gt + t + 2);
+        } else if (have_nx && g < nx.T) {
+          // the group's first tile of the next item (its Q in the other buffer)
+          if (!nq_ready) {
+            ok = lf_wait_warp(q_full0 + 8 * (qb ^ 1), ((k + 1) >> 1) & 1, abort_flag, D.status, 3);
+            nq_ready = true;
           }
-          lf_tc_fence_after();
-          issue_s(t);
-          lf_tc_commit(s_full(t & 1));
+          if (ok) ok = issue_s(nx, qb ^ 1, g, gt + it.T + g);
+          if (ok) npre |= 1u << g;
         }
-        for (int t = 0; t < it.T && ok; t++) {
-          const int g = t & 1;
-          // P(t) written and S(t) consumed by softmax group g
-          if (!lf_wait_fast(p_full(g), pc[g] & 1, abort_flag, D.status, 5)) {
-            ok = false;
-            break;
-          }
-          pc[g]++;
-          lf_tc_fence_after();
-          if (t + 2 < it.T) {
-            // the group's next scores first: they only need its S columns, now free
-            const int s2 = (gt + t + 2) % LF_TC_NS;
-            if (!lf_wait_fast(kv_full0 + 8 * s2, ((gt + t + 2) / LF_TC_NS) & 1, abort_flag,
-                              D.status, 6)) {
-              ok = false;
-              break;
-            }
-            lf_tc_fence_after();
-            issue_s(t + 2);
-            lf_tc_commit(s_full(g));
-          }
-          const int s = (gt + t) % LF_TC_NS;
-          const uint64_t dv = dv0 + (uint64_t)(s * (32768 >> 4));
-          const int ksteps = ncols(t) / 16;
-#pragma unroll
-          for (int kk = 0; kk < 8; kk++)
-            if (kk < ksteps)
-              lf_mma_ts(tmem + LF_TM_O(g), tmem + LF_TM_P(g) + 8 * kk, dv + 128 * kk, id_pv,
-                        (t >= 2 || kk > 0));
-          lf_tc_commit(kv_empty0 + 8 * s);
-          lf_tc_commit(pv_done(g));  // P columns of group g free again
-          if (t + 2 >= it.T) lf_tc_commit(o_full(g));  // group g's last tile of the item
-        }
-        if (ok) lf_tc_commit(q_empty0 + 8 * qb);  // every S of this item issued
-        k++;
-        gt += it.T;
+        if (!ok) break;
+        const int s = (gt + t) % LF_TC_NS;
+        const int ngk = (it.ng + 15) / 16 * 16;
+        const int ksteps = t < it.nband ? LF_BK / 16 : min(LF_BK, ngk - (t - it.nband) * LF_BK) / 16;
+        lf_mma_ts_phase(tmem + LF_TM_O(g), tmem + LF_TM_P(g), dv0 + (uint64_t)(s * (32768 >> 4)),
+                        2048 >> 4, id_pv, (1u << ksteps) - 1u, t >= 2 ? 1u : 0u, kv_empty0 + 8 * s,
+                        pv_done(g), t + 2 >= it.T ? o_full(g) : 0u);
       }
-      // every MMA this thread issued has completed once end_bar flips
-      lf_tc_commit(end_bar);
-      lf_wait(end_bar, 0, abort_flag, D.status, 7);
+      if (!ok) break;
+      lf_commit_w(q_empty0 + 8 * qb);  // every S of this item issued
+      k++;
+      gt += it.T;
+      idx = nidx;
+      it = nx;
+      have = have_nx;
+      pre = npre;
     }
+    // every MMA this warp issued has completed once end_bar flips
+    lf_commit_w(end_bar);
+    lf_wait_warp(end_bar, 0, abort_flag, D.status, 7);
   } else if (warp < 8) {
     // ================================================== softmax groups
     // warps 0..3 = group 0, warps 4..7 = group 1; group g takes tiles t = g, g+2, ...
@@ -534,7 +549,7 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
       }
       if (!alive) break;
       // ---- merge the two groups' partial results of this item, write O
-      const bool has_g = it.T > g, has_o = it.T > 1 - g;
+      const bool has_g = it.T > g;
       if (has_g) {
         if (!lf_wait_warp(o_full(g), oc & 1, abort_flag, D.status, 9)) {
           alive = false;

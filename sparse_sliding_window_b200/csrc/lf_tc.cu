@@ -509,21 +509,27 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
         // ---- probabilities of the tile -> P_g (TMEM) against the running
         // reference m_ref (0 until a tile says otherwise).  The tile's row sum
         // shows when the reference is off: a sum above 2^15 means some p may
-        // exceed the P format (f16) -- the row max grew; a sum below 2^-30
-        // on a row whose running sum is also that small means underflow.
-        // Either way the warp redoes the tile with the tile's own max (O_g
-        // rescaled).  S_g stays valid until this group's P is handed over.
+        // exceed the P format (f16) -- the row max grew; a sum below kLowT on
+        // a row whose running sum is also below kLowL means the tile's
+        // largest p have left the P format's precise range (f16 normals end
+        // at 2^-14, the ex2 flush at 2^-126) while they still matter to the
+        // row.  Either way the warp redoes the tile with the tile's own max
+        // (O_g rescaled).  S_g stays valid until this group's P is handed over.
         LfPvGate gate{pv_done(g), sc > 0 ? ((sc - 1) & 1) : -1, abort_flag, D.status};
         const bool any_bits = (w[0] | w[1] | w[2] | w[3]) != 0u;
         float lt = 0.f, mx = -INFINITY;
         lf_tile_pass<kF16>(tS, tP, w, sl2, m_ref, lt, mx, false, gate);
-        const bool off = any_bits && (lt > 32768.f || (lt < 9.3e-10f && l < 9.3e-10f));
+        constexpr float kLowT = kF16 ? 0.0625f : 9.3e-10f, kLowL = kF16 ? 1.f : 9.3e-10f;
+        const bool off = any_bits && (lt > 32768.f || (lt < kLowT && l < kLowL));
         if (__any_sync(0xffffffffu, off)) {
           lf_tile_pass<kF16>(tS, tP, w, sl2, m_ref, lt, mx, true, gate);  // max only
           const float ms = mx * sl2;
           const bool need = off && ms > -INFINITY;
-          const float m_new = need ? ms : m_ref;
-          const float alpha = need ? lf_ex2(m_ref - m_new) : 1.f;
+          // with nothing summed yet the reference may move anywhere; else it
+          // drops by at most 2^126 (the earlier keys, p >= 2^-126 against the
+          // old reference, then dominate), so alpha stays finite
+          const float m_new = !need ? m_ref : (l > 0.f ? fmaxf(ms, m_ref - 126.f) : ms);
+          const float alpha = (need && l > 0.f) ? lf_ex2(m_ref - m_new) : 1.f;
           l *= alpha;
           if (t >= 2 && __any_sync(0xffffffffu, need)) {
             gate.pass();

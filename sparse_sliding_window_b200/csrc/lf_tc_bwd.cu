@@ -229,65 +229,56 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
     }
   } else if (warp == 5) {
     // ================================================== MMA issuer
-    if (lane == 0) {
-      const uint64_t dr0 = lf_sdesc(sbase + LF_BW_R0, 16, 1024);
-      const uint64_t dr1 = lf_sdesc(sbase + LF_BW_R1, 16, 1024);
-      const uint64_t dc0 = lf_sdesc(sbase + LF_BW_C0(0), 16, 1024);  // K-major view
-      const uint64_t dc0mn = lf_sdesc(sbase + LF_BW_C0(0), 0, 1024);  // MN-major view
-      const uint64_t dc1 = lf_sdesc(sbase + LF_BW_C1(0), 16, 1024);
-      const uint64_t dc1mn = lf_sdesc(sbase + LF_BW_C1(0), 0, 1024);
-      const uint32_t id_acc = lf_idesc(kF16, 64, 1);
-      const int ngk = (it.ng + 15) / 16 * 16;
-      auto ncols = [&](int t) { return t < it.nband ? LF_BK : min(LF_BK, ngk - (t - it.nband) * LF_BK); };
-      auto issue_s = [&](int t) {
-        const uint64_t so = (uint64_t)((t % LF_BW_NS) * (32768 >> 4));
-        const uint32_t id = lf_idesc(kF16, ncols(t), 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++) {
-          lf_mma_ss(tmem + LF_BT_S, dr0 + 2 * kk, dc0 + so + 2 * kk, id, kk > 0);
-          lf_mma_ss(tmem + LF_BT_DP, dr1 + 2 * kk, dc1 + so + 2 * kk, id, kk > 0);
-        }
-      };
-      bool ok = lf_wait_fast(row_full, 0, abort_flag, D.status, 23) &&
-                lf_wait_fast(col_full0, 0, abort_flag, D.status, 24);
-      if (ok) {
+    // the whole warp waits; one elected lane issues each phase
+    const uint64_t dr0 = lf_sdesc(sbase + LF_BW_R0, 16, 1024);
+    const uint64_t dr1 = lf_sdesc(sbase + LF_BW_R1, 16, 1024);
+    const uint64_t dc0 = lf_sdesc(sbase + LF_BW_C0(0), 16, 1024);  // K-major view
+    const uint64_t dc0mn = lf_sdesc(sbase + LF_BW_C0(0), 0, 1024);  // MN-major view
+    const uint64_t dc1 = lf_sdesc(sbase + LF_BW_C1(0), 16, 1024);
+    const uint64_t dc1mn = lf_sdesc(sbase + LF_BW_C1(0), 0, 1024);
+    const uint32_t id_acc = lf_idesc(kF16, 64, 1);
+    const int ngk = (it.ng + 15) / 16 * 16;
+    auto ncols = [&](int t) { return t < it.nband ? LF_BK : min(LF_BK, ngk - (t - it.nband) * LF_BK); };
+    // S = R0 C0^T and dP = R1 C1^T of column tile t -> s_full
+    auto issue_s = [&](int t) {
+      const uint64_t so = (uint64_t)((t % LF_BW_NS) * (32768 >> 4));
+      lf_mma_s2_phase(tmem + LF_BT_S, dr0, dc0 + so, tmem + LF_BT_DP, dr1, dc1 + so,
+                      lf_idesc(kF16, ncols(t), 0), s_full);
+    };
+    bool ok = lf_wait_warp(row_full, 0, abort_flag, D.status, 23) &&
+              lf_wait_warp(col_full0, 0, abort_flag, D.status, 24);
+    if (ok) {
+      lf_tc_fence_after();
+      issue_s(0);
+      for (int t = 0; t < T; t++) {
+        if (!lf_wait_warp(ds_full, t & 1, abort_flag, D.status, 25)) break;
         lf_tc_fence_after();
-        issue_s(0);
-        lf_tc_commit(s_full);
-        for (int t = 0; t < T; t++) {
-          if (!lf_wait_fast(ds_full, t & 1, abort_flag, D.status, 25)) break;
+        if (t + 1 < T) {
+          const int s2 = (t + 1) % LF_BW_NS;
+          if (!lf_wait_warp(col_full0 + 8 * s2, ((t + 1) / LF_BW_NS) & 1, abort_flag, D.status, 26))
+            break;
           lf_tc_fence_after();
-          if (t + 1 < T) {
-            const int s2 = (t + 1) % LF_BW_NS;
-            if (!lf_wait_fast(col_full0 + 8 * s2, ((t + 1) / LF_BW_NS) & 1, abort_flag, D.status, 26))
-              break;
-            lf_tc_fence_after();
-            issue_s(t + 1);
-            lf_tc_commit(s_full);
-          }
-          const uint64_t so = (uint64_t)((t % LF_BW_NS) * (32768 >> 4));
-          const int ksteps = ncols(t) / 16;
-#pragma unroll
-          for (int kk = 0; kk < 8; kk++) {
-            if (kk >= ksteps) continue;
-            const uint32_t acc = (t > 0 || kk > 0);
-            if (kModeQ) {
-              // dQ += dS K   (K tile as the MN-major B operand)
-              lf_mma_ts(tmem + LF_BT_ACC0, tmem + LF_BT_A0 + 8 * kk, dc0mn + so + 128 * kk, id_acc, acc);
-            } else {
-              // dV += P^T dO ; dK += dS^T Q
-              lf_mma_ts(tmem + LF_BT_ACC0, tmem + LF_BT_A0 + 8 * kk, dc1mn + so + 128 * kk, id_acc, acc);
-              lf_mma_ts(tmem + LF_BT_ACC1, tmem + LF_BT_A1 + 8 * kk, dc0mn + so + 128 * kk, id_acc, acc);
-            }
-          }
-          lf_tc_commit(col_empty0 + 8 * (t % LF_BW_NS));
-          lf_tc_commit(acc_done);
-          if (t + 1 == T) lf_tc_commit(o_full);
+          issue_s(t + 1);
+        }
+        const uint64_t so = (uint64_t)((t % LF_BW_NS) * (32768 >> 4));
+        const uint32_t kmask = (1u << (ncols(t) / 16)) - 1u;
+        const uint32_t acc0 = t > 0 ? 1u : 0u;
+        const uint32_t last = t + 1 == T ? o_full : 0u;
+        if (kModeQ) {
+          // dQ += dS K   (K tile as the MN-major B operand)
+          lf_mma_ts_phase(tmem + LF_BT_ACC0, tmem + LF_BT_A0, dc0mn + so, 2048 >> 4, id_acc, kmask,
+                          acc0, col_empty0 + 8 * (t % LF_BW_NS), acc_done, last);
+        } else {
+          // dV += P^T dO ; dK += dS^T Q
+          lf_mma_ts_phase(tmem + LF_BT_ACC0, tmem + LF_BT_A0, dc1mn + so, 2048 >> 4, id_acc, kmask,
+                          acc0, 0u, 0u, 0u);
+          lf_mma_ts_phase(tmem + LF_BT_ACC1, tmem + LF_BT_A1, dc0mn + so, 2048 >> 4, id_acc, kmask,
+                          acc0, col_empty0 + 8 * (t % LF_BW_NS), acc_done, last);
         }
       }
-      lf_tc_commit(end_bar);
-      lf_wait(end_bar, 0, abort_flag, D.status, 27);
     }
+    lf_commit_w(end_bar);
+    lf_wait_warp(end_bar, 0, abort_flag, D.status, 27);
   } else {
     // ================================================== P / dS warps (0..3)
     const int q = warp * 32 + lane;

@@ -19,6 +19,7 @@
 // status word slots (int32 each) at the start of the workspace
 #define LF_ST_CODE 0      // first error code (atomicCAS from 0)
 #define LF_ST_DETAIL 1    // kernel-specific detail of the first error
+#define LF_ST_SCHED 2     // work-item counter of the persistent forward (zero at each call)
 #define LF_ST_WORDS 8
 
 // per-sequence info written by the mask pass (int32 each)

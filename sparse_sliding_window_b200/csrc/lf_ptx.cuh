@@ -324,12 +324,18 @@ __device__ __forceinline__ uint32_t lf_idesc(int f16, int n, int b_mn) {
 // Bits k (0..31) of the 32-column chunk starting at column `base` whose
 // column lies in [lo, hi].
 __device__ __forceinline__ uint32_t lf_range_bits(int lo, int hi, int base) {
-  int a = lo - base, z = hi - base;
-  if (z < 0 || a > 31 || a > z) return 0u;
-  a = max(a, 0);
-  z = min(z, 31);
-  const uint32_t upto = z == 31 ? 0xffffffffu : ((1u << (z + 1)) - 1u);
-  return upto & ~((1u << a) - 1u);
+  const int a = lo - base, z = hi - base;  // selects, no branches
+  const uint32_t ge = a <= 0 ? 0xffffffffu : (a > 31 ? 0u : (0xffffffffu << a));
+  const uint32_t le = z >= 31 ? 0xffffffffu : (z < 0 ? 0u : (0xffffffffu >> (31 - z)));
+  return ge & le;
+}
+
+// A value the compiler must keep in a register (it may not re-read it from
+// the kernel parameter bank at each use).
+__device__ __forceinline__ int lf_reg(int x) {
+  int y;
+  asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
 }
 
 // One pass over the 4 column chunks of a row's S tile (TMEM lane of this
@@ -351,6 +357,19 @@ __device__ __forceinline__ void lf_tmem_ld32_nowait(uint32_t taddr, uint32_t (&r
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
         "=r"(r[31])
       : "r"(taddr));
+}
+
+// Orders the use of r after an earlier tcgen05.wait::ld (no instruction).
+__device__ __forceinline__ void lf_tmem_pin_regs(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
 }
 
 __device__ __forceinline__ void lf_tmem_wait_ld_regs(uint32_t (&r)[32]) {

@@ -61,25 +61,29 @@
 #include "lf_ptx.cuh"
 #include "lf_tc.cuh"
 
-#define LF_TC_THREADS 320
-#define LF_TC_NS 5
+#define LF_TC_THREADS 384
+#define LF_TC_NS 3
 #define LF_TC_MAX_MAPS 28
 #define LF_TC_MAX_SEG 32
 
-// TMEM column map (per softmax group g = 0, 1)
-#define LF_TM_S(g) ((g)*128)
-#define LF_TM_O(g) (256 + (g)*64)
-#define LF_TM_P(g) (384 + (g)*64)
+// TMEM column map: stream g owns columns [256g, 256g + 256): its S tile,
+// O accumulator and P tile (bf16/f16 pairs, the A operand of P.V)
+#define LF_TM_S(g) ((g)*256)
+#define LF_TM_O(g) ((g)*256 + 128)
+#define LF_TM_P(g) ((g)*256 + 192)
 #define LF_TM_COLS 512
 
-// shared memory map (bytes from the 1024-aligned base): two Q buffers, then
-// LF_TC_NS stages of (K tile, V tile), barriers, the merge exchange
-#define LF_SM_Q(i) ((i)*16384)
-#define LF_SM_K(s) (32768 + (s)*32768)
-#define LF_SM_V(s) (32768 + (s)*32768 + 16384)
-#define LF_SM_BAR (32768 + LF_TC_NS * 32768)
-#define LF_SM_XCH (LF_SM_BAR + 512)
-#define LF_SMEM_BYTES (LF_SM_XCH + 2 * LF_BQ * 8)
+// shared memory map (bytes from the 1024-aligned base): per stream a Q
+// buffer and LF_TC_NS stages of (K tile, V tile); then the barriers, the
+// TMEM slot, the abort flag and the work-item slots
+#define LF_SM_STREAM (16384 + LF_TC_NS * 32768)
+#define LF_SM_Q(g) ((g)*LF_SM_STREAM)
+#define LF_SM_K(g, s) ((g)*LF_SM_STREAM + 16384 + (s)*32768)
+#define LF_SM_V(g, s) ((g)*LF_SM_STREAM + 16384 + (s)*32768 + 16384)
+#define LF_SM_BAR (2 * LF_SM_STREAM)
+#define LF_SMEM_BYTES (LF_SM_BAR + 1024)
+static_assert(96 + 16 * LF_TC_NS <= 160, "per-stream barrier block");
+static_assert(LF_SMEM_BYTES <= 232448, "shared memory per CTA");
 
 
 struct LfTcParams {
@@ -237,37 +241,39 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
   const LfDev &D = P.dev;
   const int n = D.n;
   const int nitems = P.n_gitems + D.B * P.per_batch;
+  // stream of this warp: softmax warps 0-3 / 4-7, producer 8 / 10, MMA 9 / 11
+  const int g = warp < 8 ? warp >> 2 : (warp - 8) >> 1;
 
-  // barriers (8 bytes each)
-  const uint32_t bar = sbase + LF_SM_BAR;
-  const uint32_t q_full0 = bar, q_empty0 = bar + 16, kv_full0 = bar + 32,
-                 kv_empty0 = bar + 32 + 8 * LF_TC_NS;
-  const uint32_t gb0 = bar + 32 + 16 * LF_TC_NS;  // per-group barriers, 5 x 2
-  auto s_full = [&](int g) { return gb0 + 8 * g; };
-  auto p_full = [&](int g) { return gb0 + 16 + 8 * g; };
-  auto pv_done = [&](int g) { return gb0 + 32 + 8 * g; };
-  auto o_full = [&](int g) { return gb0 + 48 + 8 * g; };
-  const uint32_t mrg0 = gb0 + 64, mrg1 = gb0 + 72, end_bar = gb0 + 80;
-  uint32_t *tmem_slot = (uint32_t *)(gbase + LF_SM_BAR + 448);
-  volatile int *abort_flag = (volatile int *)(gbase + LF_SM_BAR + 452);
-  float2 *xch = (float2 *)(gbase + LF_SM_XCH);  // [2][128] (max, sum) per group and row
+  // barriers of stream g (8 bytes each, 12 + 2 LF_TC_NS per stream, 160-byte stride)
+  const uint32_t bar = sbase + LF_SM_BAR + 160 * g;
+  const uint32_t q_full = bar, q_empty = bar + 8, s_full = bar + 16, p_full = bar + 24,
+                 pv_done = bar + 32, o_full = bar + 40, o_free = bar + 48, end_bar = bar + 56;
+  const uint32_t it_full0 = bar + 64, it_empty0 = bar + 80, kv_full0 = bar + 96,
+                 kv_empty0 = bar + 96 + 8 * LF_TC_NS;
+  uint32_t *tmem_slot = (uint32_t *)(gbase + LF_SM_BAR + 512);
+  volatile int *abort_flag = (volatile int *)(gbase + LF_SM_BAR + 516);
+  volatile int *item_slot = (volatile int *)(gbase + LF_SM_BAR + 520) + 2 * g;  // [2] per stream
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; i++) {
-      lf_mbar_init(q_full0 + 8 * i, 1);
-      lf_mbar_init(q_empty0 + 8 * i, 1);
-      lf_mbar_init(s_full(i), 1);
-      lf_mbar_init(p_full(i), 4);
-      lf_mbar_init(pv_done(i), 1);
-      lf_mbar_init(o_full(i), 1);
+    for (int gg = 0; gg < 2; gg++) {
+      const uint32_t b0 = sbase + LF_SM_BAR + 160 * gg;
+      lf_mbar_init(b0, 1);       // q_full
+      lf_mbar_init(b0 + 8, 1);   // q_empty
+      lf_mbar_init(b0 + 16, 1);  // s_full
+      lf_mbar_init(b0 + 24, 4);  // p_full (four softmax warps)
+      lf_mbar_init(b0 + 32, 1);  // pv_done
+      lf_mbar_init(b0 + 40, 1);  // o_full
+      lf_mbar_init(b0 + 48, 4);  // o_free (four softmax warps)
+      lf_mbar_init(b0 + 56, 1);  // end
+      for (int i = 0; i < 2; i++) {
+        lf_mbar_init(b0 + 64 + 8 * i, 1);  // item slot filled
+        lf_mbar_init(b0 + 80 + 8 * i, 5);  // item slot read (MMA warp + four softmax warps)
+      }
+      for (int s = 0; s < LF_TC_NS; s++) {
+        lf_mbar_init(b0 + 96 + 8 * s, 1);
+        lf_mbar_init(b0 + 96 + 8 * LF_TC_NS + 8 * s, 1);
+      }
     }
-    for (int s = 0; s < LF_TC_NS; s++) {
-      lf_mbar_init(kv_full0 + 8 * s, 1);
-      lf_mbar_init(kv_empty0 + 8 * s, 1);
-    }
-    lf_mbar_init(mrg0, 8);
-    lf_mbar_init(mrg1, 8);
-    lf_mbar_init(end_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -284,21 +290,50 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
   lf_tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
-    // ================================================== TMA producer
+  // consumers take the stream's items from its two slots in order; -1 ends
+  auto take_item = [&](int k, int &idx) -> bool {
+    const int slot = k & 1;
+    if (!lf_wait_warp(it_full0 + 8 * slot, (k >> 1) & 1, abort_flag, D.status, 15)) return false;
+    idx = item_slot[slot];
+    __syncwarp();
+    if (lane == 0) lf_mbar_arrive(it_empty0 + 8 * slot);
+    return true;
+  };
+
+  if (warp == 8 || warp == 10) {
+    // ================================================== TMA producer + scheduler
     if (lane == 0) {
       int gt = 0, k = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < nitems && ok; idx += gridDim.x) {
+      while (ok) {
+        // next work item of the whole grid (largest first: global rows, then
+        // band blocks); empty items are skipped
+        int idx;
         LfItem it;
-        if (!lf_decode(P, idx, it)) continue;
-        const int qb = k & 1;
-        if (k >= 2 && !lf_wait_fast(q_empty0 + 8 * qb, ((k >> 1) & 1) ^ 1, abort_flag, D.status, 1)) {
+        for (;;) {
+          idx = atomicAdd(D.status + LF_ST_SCHED, 1);
+          if (idx >= nitems) {
+            idx = -1;
+            break;
+          }
+          if (lf_decode(P, idx, it)) break;
+        }
+        const int slot = k & 1;
+        if (k >= 2 &&
+            !lf_wait_fast(it_empty0 + 8 * slot, ((k >> 1) & 1) ^ 1, abort_flag, D.status, 16)) {
           ok = false;
           break;
         }
-        lf_mbar_expect_tx(q_full0 + 8 * qb, 16384);
-        lf_tma_load4(sbase + LF_SM_Q(qb), &P.maps[it.mq], q_full0 + 8 * qb, 0, it.qrow0, it.h, it.b);
+        item_slot[slot] = idx;
+        lf_mbar_arrive(it_full0 + 8 * slot);
+        if (idx < 0) break;
+        // the previous item's scores all computed: Q may be replaced
+        if (k >= 1 && !lf_wait_fast(q_empty, (k - 1) & 1, abort_flag, D.status, 1)) {
+          ok = false;
+          break;
+        }
+        lf_mbar_expect_tx(q_full, 16384);
+        lf_tma_load4(sbase + LF_SM_Q(g), &P.maps[it.mq], q_full, 0, it.qrow0, it.h, it.b);
         const int tk0 = it.qrow0 - D.r;
         for (int t = 0; t < it.T; t++, gt++) {
           const int s = gt % LF_TC_NS;
@@ -322,8 +357,8 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
             bytes = 2 * P.gbox * 128;
           }
           lf_mbar_expect_tx(kv_full0 + 8 * s, bytes);
-          lf_tma_load4(sbase + LF_SM_K(s), km, kv_full0 + 8 * s, 0, row, it.h, it.b);
-          lf_tma_load4(sbase + LF_SM_V(s), vm, kv_full0 + 8 * s, 0, row, it.h, it.b);
+          lf_tma_load4(sbase + LF_SM_K(g, s), km, kv_full0 + 8 * s, 0, row, it.h, it.b);
+          lf_tma_load4(sbase + LF_SM_V(g, s), vm, kv_full0 + 8 * s, 0, row, it.h, it.b);
         }
         k++;
       }
@@ -333,152 +368,144 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
           lf_wait(kv_full0 + 8 * (i % LF_TC_NS), (i / LF_TC_NS) & 1, abort_flag, D.status, 11);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 9 || warp == 11) {
     // ================================================== MMA issuer
-    // The whole warp walks the tile stream and waits together; one elected
-    // lane issues each MMA phase.  Order per tile t of group g = t & 1:
-    // wait P_g(t), issue the group's next S (tile t + 2, or at the end of
-    // the item the group's first tile of the next item, so the softmax
-    // finds it ready after the merge), then O_g += P_g V_t.
-    const uint64_t dq0 = lf_sdesc(sbase + LF_SM_Q(0), 16, 1024);
-    const uint64_t dk0 = lf_sdesc(sbase + LF_SM_K(0), 16, 1024);
-    const uint64_t dv0 = lf_sdesc(sbase + LF_SM_V(0), 0, 1024);
+    // The whole warp waits; one elected lane issues each phase.  Per tile t
+    // of an item: wait P(t), issue S(t + 1) (S is free once P(t) is
+    // written), then O (+)= P(t) V_t.
+    const uint64_t dq0 = lf_sdesc(sbase + LF_SM_Q(g), 16, 1024);
+    const uint64_t dk0 = lf_sdesc(sbase + LF_SM_K(g, 0), 16, 1024);
+    const uint64_t dv0 = lf_sdesc(sbase + LF_SM_V(g, 0), 0, 1024);
     const uint32_t id_pv = lf_idesc(kF16, 64, 1);
     int gt = 0, k = 0;
-    uint32_t pc = 0;  // bit g: parity of group g's next p_full phase
     bool ok = true;
-    // S of tile t of item `it` (Q buffer qb, ring position gtt) into S_g
-    auto issue_s = [&](const LfItem &it, int qb, int t, int gtt) -> bool {
-      const int s = gtt % LF_TC_NS;
-      if (!lf_wait_warp(kv_full0 + 8 * s, (gtt / LF_TC_NS) & 1, abort_flag, D.status, 4)) return false;
-      lf_tc_fence_after();
-      const int ngk = (it.ng + 15) / 16 * 16;  // global key tile width, multiple of 16
-      const int nc = t < it.nband ? LF_BK : min(LF_BK, ngk - (t - it.nband) * LF_BK);
-      lf_mma_s_phase(tmem + LF_TM_S(t & 1), dq0 + (uint64_t)(qb * (16384 >> 4)),
-                     dk0 + (uint64_t)(s * (32768 >> 4)), lf_idesc(kF16, nc, 0), s_full(t & 1));
-      return true;
-    };
-    int idx = blockIdx.x;
-    LfItem it;
-    bool have = false;
-    for (; idx < nitems; idx += gridDim.x)
-      if (lf_decode(P, idx, it)) {
-        have = true;
-        break;
-      }
-    uint32_t pre = 0;  // bit t: S of tile t (< 2) of `it` already issued
-    while (have && ok) {
-      const int qb = k & 1;
-      if (!lf_wait_warp(q_full0 + 8 * qb, (k >> 1) & 1, abort_flag, D.status, 3)) {
+    while (ok) {
+      int idx;
+      if (!take_item(k, idx)) {
         ok = false;
         break;
       }
-      for (int t = 0; t < 2 && t < it.T && ok; t++)
-        if (!((pre >> t) & 1u)) ok = issue_s(it, qb, t, gt + t);
-      if (!ok) break;
-      // the next item of this CTA
-      LfItem nx;
-      bool have_nx = false;
-      int nidx = idx + gridDim.x;
-      for (; nidx < nitems; nidx += gridDim.x)
-        if (lf_decode(P, nidx, nx)) {
-          have_nx = true;
-          break;
-        }
-      uint32_t npre = 0;
-      bool nq_ready = false;
+      if (idx < 0) break;
+      LfItem it;
+      lf_decode(P, idx, it);
+      const int ngk = (it.ng + 15) / 16 * 16;  // global key tile width, multiple of 16
+      auto ncols = [&](int t) { return t < it.nband ? LF_BK : min(LF_BK, ngk - (t - it.nband) * LF_BK); };
+      auto issue_s = [&](int t) -> bool {
+        const int j = gt + t, s = j % LF_TC_NS;
+        if (!lf_wait_warp(kv_full0 + 8 * s, (j / LF_TC_NS) & 1, abort_flag, D.status, 4)) return false;
+        lf_tc_fence_after();
+        lf_mma_s_phase(tmem + LF_TM_S(g), dq0, dk0 + (uint64_t)(s * (32768 >> 4)),
+                       lf_idesc(kF16, ncols(t), 0), s_full);
+        if (t + 1 == it.T) lf_commit_w(q_empty);  // every S of the item issued
+        return true;
+      };
+      if (!lf_wait_warp(q_full, k & 1, abort_flag, D.status, 3)) {
+        ok = false;
+        break;
+      }
+      if (!issue_s(0)) {
+        ok = false;
+        break;
+      }
       for (int t = 0; t < it.T && ok; t++) {
-        const int g = t & 1;
-        // P(t) written and S(t) consumed by softmax group g
-        if (!lf_wait_warp(p_full(g), (pc >> g) & 1u, abort_flag, D.status, 5)) {
+        const int j = gt + t;
+        // P(t) written and S(t) consumed by the softmax warps
+        if (!lf_wait_warp(p_full, j & 1, abort_flag, D.status, 5)) {
           ok = false;
           break;
         }
-        pc ^= 1u << g;
         lf_tc_fence_after();
-        if (t + 2 < it.T) {
-          ok = issue_s(it, qb, t + 2, gt + t + 2);
-        } else if (have_nx && g < nx.T) {
-          // the group's first tile of the next item (its Q in the other buffer)
-          if (!nq_ready) {
-            ok = lf_wait_warp(q_full0 + 8 * (qb ^ 1), ((k + 1) >> 1) & 1, abort_flag, D.status, 3);
-            nq_ready = true;
-          }
-          if (ok) ok = issue_s(nx, qb ^ 1, g, gt + it.T + g);
-          if (ok) npre |= 1u << g;
+        if (t + 1 < it.T && !issue_s(t + 1)) {
+          ok = false;
+          break;
         }
-        if (!ok) break;
-        const int s = (gt + t) % LF_TC_NS;
-        const int ngk = (it.ng + 15) / 16 * 16;
-        const int ksteps = t < it.nband ? LF_BK / 16 : min(LF_BK, ngk - (t - it.nband) * LF_BK) / 16;
+        // O read out by the softmax warps at the end of the previous item
+        if (t == 0 && k >= 1 && !lf_wait_warp(o_free, (k - 1) & 1, abort_flag, D.status, 6)) {
+          ok = false;
+          break;
+        }
+        const int s = j % LF_TC_NS;
         lf_mma_ts_phase(tmem + LF_TM_O(g), tmem + LF_TM_P(g), dv0 + (uint64_t)(s * (32768 >> 4)),
-                        2048 >> 4, id_pv, (1u << ksteps) - 1u, t >= 2 ? 1u : 0u, kv_empty0 + 8 * s,
-                        pv_done(g), t + 2 >= it.T ? o_full(g) : 0u);
+                        2048 >> 4, id_pv, (1u << (ncols(t) / 16)) - 1u, t > 0 ? 1u : 0u,
+                        kv_empty0 + 8 * s, pv_done, t + 1 == it.T ? o_full : 0u);
       }
-      if (!ok) break;
-      lf_commit_w(q_empty0 + 8 * qb);  // every S of this item issued
       k++;
       gt += it.T;
-      idx = nidx;
-      it = nx;
-      have = have_nx;
-      pre = npre;
     }
     // every MMA this warp issued has completed once end_bar flips
     lf_commit_w(end_bar);
     lf_wait_warp(end_bar, 0, abort_flag, D.status, 7);
   } else if (warp < 8) {
-    // ================================================== softmax groups
-    // warps 0..3 = group 0, warps 4..7 = group 1; group g takes tiles t = g, g+2, ...
-    const int g = warp >> 2;
+    // ================================================== softmax warps
+    // warps 4g .. 4g+3 of stream g: one TMEM lane = one query row per thread
     const int quarter = warp & 3;
     const int q = quarter * 32 + lane;  // query row of the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + LF_TM_S(g), tP = tmem + lane_off + LF_TM_P(g);
     const uint32_t tO = tmem + lane_off + LF_TM_O(g);
     const float sl2 = D.scale_log2;
-    int sc = 0, oc = 0, k = 0;
-    bool alive = true;
-    for (int idx = blockIdx.x; idx < nitems && alive; idx += gridDim.x) {
+    // loop-invariant parameters held in registers (not re-read from the
+    // parameter bank inside the tile loop)
+    const int rr = lf_reg(D.r), causal = lf_reg(D.causal);
+    // per-row context of a work item: taken, decoded and its global loads
+    // issued before the previous item's epilogue, which hides their latency
+    struct Ctx {
       LfItem it;
-      if (!lf_decode(P, idx, it)) continue;
-      const int32_t *mrow = D.mask + (size_t)it.b * n;
-      const int32_t *gl = D.gidx + (size_t)it.b * D.G;
-      int code = 0, pos = 0;
-      bool active;
-      if (it.gitem) {
-        active = it.qrow0 + q < it.ng;
+      int code, pos, e_lo, e_hi;
+      bool active, padded;
+    };
+    auto setup = [&](int kk, Ctx &c) -> int {  // 1: item, 0: no more items, -1: aborted
+      int idx;
+      if (!take_item(kk, idx)) return -1;
+      if (idx < 0) return 0;
+      lf_decode(P, idx, c.it);
+      const int32_t *mr = D.mask + (size_t)c.it.b * n;
+      c.code = 0;
+      c.pos = 0;
+      if (c.it.gitem) {
+        c.active = c.it.qrow0 + q < c.it.ng;
       } else {
-        const int t = it.qrow0 + q;
-        if (t < it.cnt) {
-          pos = it.rho + t * it.d;
-          code = mrow[pos];
+        const int t = c.it.qrow0 + q;
+        if (t < c.it.cnt) {
+          c.pos = c.it.rho + t * c.it.d;
+          c.code = mr[c.pos];
         }
-        active = (code == 1);
+        c.active = (c.code == 1);
       }
-      const bool padded = D.binfo[(size_t)it.b * LF_BI_WORDS + LF_BI_NVALID] < n;
+      c.padded = D.binfo[(size_t)c.it.b * LF_BI_WORDS + LF_BI_NVALID] < n;
       // global keys already in the row's window: index range [e_lo, e_hi) of
       // the sorted global list, from the rank array (filtered by residue)
-      int e_lo = 0, e_hi = 0;
-      if (!it.gitem && it.nglob > 0 && active) {
-        const int32_t *gr = D.grank + (size_t)it.b * (n + 1);
-        e_lo = gr[max(pos - D.r * it.d, 0)];
-        e_hi = gr[min((D.causal ? pos : pos + D.r * it.d) + 1, n)];
+      c.e_lo = 0;
+      c.e_hi = 0;
+      if (!c.it.gitem && c.it.nglob > 0 && c.active) {
+        const int32_t *gr = D.grank + (size_t)c.it.b * (n + 1);
+        c.e_lo = gr[max(c.pos - rr * c.it.d, 0)];
+        c.e_hi = gr[min((causal ? c.pos : c.pos + rr * c.it.d) + 1, n)];
       }
-      const int tk0 = it.qrow0 - D.r;
+      return 1;
+    };
+    int gt = 0, k = 0;
+    bool alive = true;
+    Ctx cur;
+    int st = setup(0, cur);
+    alive = st >= 0;
+    while (st == 1) {
+      const LfItem &it = cur.it;
+      const int code = cur.code, pos = cur.pos, e_lo = cur.e_lo, e_hi = cur.e_hi;
+      const bool active = cur.active, padded = cur.padded;
+      const int32_t *mrow = D.mask + (size_t)it.b * n;
+      const int32_t *gl = D.gidx + (size_t)it.b * D.G;
+      const int tk0 = it.qrow0 - rr;
       float m_ref = 0.f, l = 0.f;
-      for (int t = g; t < it.T; t += 2) {
-        if (!lf_wait_warp(s_full(g), sc & 1, abort_flag, D.status, 8)) {
-          alive = false;
-          break;
-        }
-        lf_tc_fence_after();
-        // ---- attend mask of row q over the tile's 128 columns (4 words)
+      for (int t = 0; t < it.T; t++) {
+        const int j = gt + t;
+        // ---- attend mask of row q over the tile's 128 columns (4 words);
+        // computed while the tile's scores are still on their way
         uint32_t w[4];
         if (t < it.nband) {
           const int kb = it.gitem ? (it.kt0 + t) * LF_BK : tk0 + t * LF_BK;
           int lo = 0, hi = LF_BK - 1;
-          if (!it.gitem) lf_band_cols(q, t, D.r, D.causal, lo, hi);
+          if (!it.gitem) lf_band_cols(q, t, rr, causal, lo, hi);
           lo = max(lo, -kb);  // keys exist on [0, cnt)
           hi = min(hi, it.cnt - 1 - kb);
           if (!active) hi = -1;
@@ -506,7 +533,12 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
             w[cc] = lf_range_bits(0, hi, 32 * cc) & ~inwin;
           }
         }
-        // ---- probabilities of the tile -> P_g (TMEM) against the running
+        if (!lf_wait_warp(s_full, j & 1, abort_flag, D.status, 8)) {
+          alive = false;
+          break;
+        }
+        lf_tc_fence_after();
+        // ---- probabilities of the tile -> P (TMEM) against the running
         // reference m_ref (0 until a tile says otherwise).  The tile's row sum
         // shows when the reference is off: a sum above 2^15 means some p may
         // exceed the P format (f16) -- the row max grew; a sum below kLowT on
@@ -514,8 +546,8 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
         // largest p have left the P format's precise range (f16 normals end
         // at 2^-14, the ex2 flush at 2^-126) while they still matter to the
         // row.  Either way the warp redoes the tile with the tile's own max
-        // (O_g rescaled).  S_g stays valid until this group's P is handed over.
-        LfPvGate gate{pv_done(g), sc > 0 ? ((sc - 1) & 1) : -1, abort_flag, D.status};
+        // (O rescaled).  P(t - 1) must have been consumed before P is written.
+        LfPvGate gate{pv_done, j > 0 ? (j - 1) & 1 : -1, abort_flag, D.status};
         const bool any_bits = (w[0] | w[1] | w[2] | w[3]) != 0u;
         float lt = 0.f, mx = -INFINITY;
         lf_tile_pass<kF16>(tS, tP, w, sl2, m_ref, lt, mx, false, gate);
@@ -531,8 +563,8 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
           const float m_new = !need ? m_ref : (l > 0.f ? fmaxf(ms, m_ref - 126.f) : ms);
           const float alpha = (need && l > 0.f) ? lf_ex2(m_ref - m_new) : 1.f;
           l *= alpha;
-          if (t >= 2 && __any_sync(0xffffffffu, need)) {
-            gate.pass();
+          if (t >= 1 && __any_sync(0xffffffffu, need)) {
+            gate.pass();  // O holds P.V of the item's earlier tiles, all done
 #pragma unroll
             for (int half = 0; half < 2; half++) {
               float ov[32];
@@ -547,104 +579,77 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
         }
         l += lt;
         gate.pass();  // (no-op unless every chunk of the tile was skipped)
-        sc++;
         lf_tmem_wait_st();
         lf_tc_fence_before();
         __syncwarp();
-        if (lane == 0) lf_mbar_arrive(p_full(g));
+        if (lane == 0) lf_mbar_arrive(p_full);
       }
       if (!alive) break;
-      // ---- merge the two groups' partial results of this item, write O
-      const bool has_g = it.T > g;
-      if (has_g) {
-        if (!lf_wait_warp(o_full(g), oc & 1, abort_flag, D.status, 9)) {
-          alive = false;
-          break;
-        }
-        oc++;
+      Ctx nxt;
+      const int nst = setup(k + 1, nxt);
+      if (nst < 0) {
+        alive = false;
+        break;
       }
-      xch[g * LF_BQ + q] = make_float2(m_ref, l);
-      __syncwarp();
-      if (lane == 0) lf_mbar_arrive(mrg0);
-      if (!lf_wait_warp(mrg0, k & 1, abort_flag, D.status, 12)) {
+      // ---- item epilogue: O / l and the log-normaliser
+      if (!lf_wait_warp(o_full, k & 1, abort_flag, D.status, 9)) {
         alive = false;
         break;
       }
       lf_tc_fence_after();
-      const float2 me = xch[g * LF_BQ + q], ot = xch[(1 - g) * LF_BQ + q];
-      const float mA = g == 0 ? me.x : ot.x, lA = g == 0 ? me.y : ot.y;
-      const float mB = g == 0 ? ot.x : me.x, lB = g == 0 ? ot.y : me.y;
-      const bool hasA = it.T > 0, hasB = it.T > 1;
-      // reference of the merged row: the larger of the groups that summed anything
-      const float M = (lA > 0.f && lB > 0.f) ? fmaxf(mA, mB) : (lA > 0.f ? mA : (lB > 0.f ? mB : 0.f));
-      const float fA = (!hasA || lA <= 0.f) ? 0.f : lf_ex2(mA - M);
-      const float fB = (!hasB || lB <= 0.f) ? 0.f : lf_ex2(mB - M);
-      const float L = lA * fA + lB * fB;
-      // this group writes head-dim columns [32g, 32g + 32), 16 at a time
-      const size_t bh = (size_t)it.b * D.H + it.h;
-      const bool store_row = it.gitem ? active : (it.qrow0 + q < it.cnt && code != 2);
-      const float inv = (!it.gitem && code == 1 && L > 0.f) ? 1.f / L : (it.gitem ? 1.f : 0.f);
-      const float ca = fA * inv, cb = fB * inv;
-      size_t pi = 0, orow = 0;
-      if (it.gitem) pi = (bh * D.G + (it.qrow0 + q)) * D.nch + (it.kt0 / D.chunk_tiles);
-      else orow = bh * n + pos;
-#pragma unroll
-      for (int hh = 0; hh < 2; hh++) {
-        const int c0 = 32 * g + 16 * hh;
-        uint32_t ra[16], rb[16];
-        asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-                     : "=r"(ra[0]), "=r"(ra[1]), "=r"(ra[2]), "=r"(ra[3]), "=r"(ra[4]), "=r"(ra[5]), "=r"(ra[6]), "=r"(ra[7]),
-                       "=r"(ra[8]), "=r"(ra[9]), "=r"(ra[10]), "=r"(ra[11]), "=r"(ra[12]), "=r"(ra[13]), "=r"(ra[14]), "=r"(ra[15])
-                     : "r"(tmem + lane_off + LF_TM_O(0) + c0));
-        if (hasB)
-          asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-                       : "=r"(rb[0]), "=r"(rb[1]), "=r"(rb[2]), "=r"(rb[3]), "=r"(rb[4]), "=r"(rb[5]), "=r"(rb[6]), "=r"(rb[7]),
-                         "=r"(rb[8]), "=r"(rb[9]), "=r"(rb[10]), "=r"(rb[11]), "=r"(rb[12]), "=r"(rb[13]), "=r"(rb[14]), "=r"(rb[15])
-                       : "r"(tmem + lane_off + LF_TM_O(1) + c0));
-        asm volatile("tcgen05.wait::ld.sync.aligned;"
-                     : "+r"(ra[0]), "+r"(ra[1]), "+r"(ra[2]), "+r"(ra[3]), "+r"(ra[4]), "+r"(ra[5]), "+r"(ra[6]), "+r"(ra[7]),
-                       "+r"(ra[8]), "+r"(ra[9]), "+r"(ra[10]), "+r"(ra[11]), "+r"(ra[12]), "+r"(ra[13]), "+r"(ra[14]), "+r"(ra[15]),
-                       "+r"(rb[0]), "+r"(rb[1]), "+r"(rb[2]), "+r"(rb[3]), "+r"(rb[4]), "+r"(rb[5]), "+r"(rb[6]), "+r"(rb[7]),
-                       "+r"(rb[8]), "+r"(rb[9]), "+r"(rb[10]), "+r"(rb[11]), "+r"(rb[12]), "+r"(rb[13]), "+r"(rb[14]), "+r"(rb[15])
-                     :
-                     : "memory");
-        float v[16];
-#pragma unroll
-        for (int kk = 0; kk < 16; kk++)
-          v[kk] = __uint_as_float(ra[kk]) * ca + (hasB ? __uint_as_float(rb[kk]) * cb : 0.f);
-        if (store_row) {
-          if (it.gitem) {
-            float4 *dst = reinterpret_cast<float4 *>(P.part_acc + pi * LF_HD + c0);
-#pragma unroll
-            for (int kk = 0; kk < 4; kk++)
-              dst[kk] = make_float4(v[4 * kk], v[4 * kk + 1], v[4 * kk + 2], v[4 * kk + 3]);
-          } else {
-            uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(P.o) + orow * LF_HD + c0);
-#pragma unroll
-            for (int kk = 0; kk < 2; kk++) {
-              uint4 u;
-              u.x = lf_pack2<kF16>(v[8 * kk + 0], v[8 * kk + 1]);
-              u.y = lf_pack2<kF16>(v[8 * kk + 2], v[8 * kk + 3]);
-              u.z = lf_pack2<kF16>(v[8 * kk + 4], v[8 * kk + 5]);
-              u.w = lf_pack2<kF16>(v[8 * kk + 6], v[8 * kk + 7]);
-              dst[kk] = u;
-            }
-          }
-        }
-      }
-      if (store_row && g == 0) {
-        if (it.gitem) P.part_ml[pi] = make_float2(M, L);
-        else if (P.lse) P.lse[orow] = code == 1 ? (M + __log2f(L)) * LF_LN2 : -INFINITY;
-      }
-      // both groups finished reading O before the next item's P.V overwrites it
+      uint32_t ra[32], rb[32];
+      lf_tmem_ld32_nowait(tO, ra);
+      lf_tmem_ld32_nowait(tO + 32, rb);
+      lf_tmem_wait_ld_regs(ra);
+      lf_tmem_pin_regs(rb);
+      // O fully read: the stream's next item may overwrite it
       lf_tc_fence_before();
       __syncwarp();
-      if (lane == 0) lf_mbar_arrive(mrg1);
-      if (!lf_wait_warp(mrg1, k & 1, abort_flag, D.status, 13)) {
-        alive = false;
-        break;
+      if (lane == 0) lf_mbar_arrive(o_free);
+      const size_t bh = (size_t)it.b * D.H + it.h;
+      const bool store_row = it.gitem ? active : (it.qrow0 + q < it.cnt && code != 2);
+      if (store_row) {
+        if (it.gitem) {
+          const size_t pi = (bh * D.G + (it.qrow0 + q)) * D.nch + (it.kt0 / D.chunk_tiles);
+          float4 *dst = reinterpret_cast<float4 *>(P.part_acc + pi * LF_HD);
+#pragma unroll
+          for (int kk = 0; kk < 8; kk++)
+            dst[kk] = make_float4(__uint_as_float(ra[4 * kk]), __uint_as_float(ra[4 * kk + 1]),
+                                  __uint_as_float(ra[4 * kk + 2]), __uint_as_float(ra[4 * kk + 3]));
+#pragma unroll
+          for (int kk = 0; kk < 8; kk++)
+            dst[8 + kk] = make_float4(__uint_as_float(rb[4 * kk]), __uint_as_float(rb[4 * kk + 1]),
+                                      __uint_as_float(rb[4 * kk + 2]), __uint_as_float(rb[4 * kk + 3]));
+          P.part_ml[pi] = make_float2(m_ref, l);
+        } else {
+          const float inv = (code == 1 && l > 0.f) ? 1.f / l : 0.f;
+          const size_t orow = bh * n + pos;
+          uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(P.o) + orow * LF_HD);
+#pragma unroll
+          for (int kk = 0; kk < 4; kk++) {
+            uint4 u;
+            u.x = lf_pack2<kF16>(__uint_as_float(ra[8 * kk + 0]) * inv, __uint_as_float(ra[8 * kk + 1]) * inv);
+            u.y = lf_pack2<kF16>(__uint_as_float(ra[8 * kk + 2]) * inv, __uint_as_float(ra[8 * kk + 3]) * inv);
+            u.z = lf_pack2<kF16>(__uint_as_float(ra[8 * kk + 4]) * inv, __uint_as_float(ra[8 * kk + 5]) * inv);
+            u.w = lf_pack2<kF16>(__uint_as_float(ra[8 * kk + 6]) * inv, __uint_as_float(ra[8 * kk + 7]) * inv);
+            dst[kk] = u;
+          }
+#pragma unroll
+          for (int kk = 0; kk < 4; kk++) {
+            uint4 u;
+            u.x = lf_pack2<kF16>(__uint_as_float(rb[8 * kk + 0]) * inv, __uint_as_float(rb[8 * kk + 1]) * inv);
+            u.y = lf_pack2<kF16>(__uint_as_float(rb[8 * kk + 2]) * inv, __uint_as_float(rb[8 * kk + 3]) * inv);
+            u.z = lf_pack2<kF16>(__uint_as_float(rb[8 * kk + 4]) * inv, __uint_as_float(rb[8 * kk + 5]) * inv);
+            u.w = lf_pack2<kF16>(__uint_as_float(rb[8 * kk + 6]) * inv, __uint_as_float(rb[8 * kk + 7]) * inv);
+            dst[4 + kk] = u;
+          }
+          if (P.lse) P.lse[orow] = code == 1 ? (m_ref + __log2f(l)) * LF_LN2 : -INFINITY;
+        }
       }
       k++;
+      gt += it.T;
+      cur = nxt;
+      st = nst;
     }
   }
 

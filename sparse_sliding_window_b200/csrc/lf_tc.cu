@@ -91,6 +91,7 @@ struct LfTcParams {
   LfDev dev;
   LfTcSeg seg[LF_TC_MAX_SEG];
   int nseg, per_batch, n_gitems, ngq, gbox;
+  int sched_cta;  // 1: per-CTA item lists, 0: one grid-wide item counter
   int map_kg, map_vg, map_qgc, map_ksc, map_vsc;
   int f16;
   void *o;
@@ -253,6 +254,7 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
   uint32_t *tmem_slot = (uint32_t *)(gbase + LF_SM_BAR + 512);
   volatile int *abort_flag = (volatile int *)(gbase + LF_SM_BAR + 516);
   volatile int *item_slot = (volatile int *)(gbase + LF_SM_BAR + 520) + 2 * g;  // [2] per stream
+  int *cta_next = (int *)(gbase + LF_SM_BAR + 544);  // the CTA's next work item, shared by its streams
 
   if (threadIdx.x == 0) {
     for (int gg = 0; gg < 2; gg++) {
@@ -275,6 +277,7 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
       }
     }
     *abort_flag = 0;
+    *cta_next = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -306,12 +309,17 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
       int gt = 0, k = 0;
       bool ok = true;
       while (ok) {
-        // next work item of the whole grid (largest first: global rows, then
-        // band blocks); empty items are skipped
+        // next work item (largest first: global rows, then band blocks);
+        // empty items are skipped.  With many items per CTA they come from
+        // one grid-wide counter (balance over the whole grid); with a few,
+        // each CTA walks its own list blockIdx.x, blockIdx.x + gridDim.x, ...,
+        // taken by whichever of its two streams is free -- so a CTA's last
+        // item mostly runs alone instead of two late items sharing an SM.
         int idx;
         LfItem it;
         for (;;) {
-          idx = atomicAdd(D.status + LF_ST_SCHED, 1);
+          idx = P.sched_cta ? blockIdx.x + gridDim.x * atomicAdd(cta_next, 1)
+                            : atomicAdd(D.status + LF_ST_SCHED, 1);
           if (idx >= nitems) {
             idx = -1;
             break;
@@ -875,6 +883,7 @@ int lf_tc_fwd(const LfLaunch &L, const LfTcArgs &a, char *err, size_t errlen) {
         nsm = 148;
     }
     const unsigned grid = (unsigned)std::min<long long>(items, nsm);  // persistent: one CTA per SM
+    P.sched_cta = items <= 4LL * grid ? 1 : 0;
     if (a.ev_start && a.ev_stop) cudaEventRecord(a.ev_start, L.stream);
     kern<<<grid, LF_TC_THREADS, LF_SMEM_BYTES, L.stream>>>(P);
     lf_launches_add(1);

@@ -187,15 +187,17 @@ extern "C" int lf_attn_fwd(const lf_attn_params *p, const void *q_s, const void 
     return st;
   LfLaunch L;
   if ((st = lf_bind_ws(p, 0, workspace, ws_bytes, mask, stream, L))) return st;
-  if ((st = lf_cuda(lf_launch_mask_pass(L), "mask pass"))) return st;
   const bool tc = p->dtype != LF_F32 && p->kernel != LF_KERNEL_SIMT;
   if (tc) {
+    // the tensor-core path launches the mask pass itself (fused with its gather)
     LfTcArgs a{q_s, k_s, v_s, q_g, k_g, v_g, o, lse, g_ev_start, g_ev_stop};
     st = lf_tc_fwd(L, a, g_err, sizeof(g_err));
     if (st == LF_ERR_UNSUPPORTED && p->kernel == LF_KERNEL_AUTO) {
-      // shape outside the tensor-core kernel's parameter block: CUDA-core kernel
+      // shape outside the tensor-core kernel's parameter block (refused before
+      // any launch): CUDA-core kernel
       g_err[0] = 0;
       st = LF_OK;
+      if ((st = lf_cuda(lf_launch_mask_pass(L), "mask pass"))) return st;
       if (g_ev_start && g_ev_stop) cudaEventRecord(g_ev_start, L.stream);
       if ((st = lf_cuda(lf_launch_simt_fwd(L, q_s, k_s, v_s, q_g, k_g, v_g, o, lse), "forward")))
         return st;
@@ -203,6 +205,7 @@ extern "C" int lf_attn_fwd(const lf_attn_params *p, const void *q_s, const void 
     }
     if (st) return st;
   } else {
+    if ((st = lf_cuda(lf_launch_mask_pass(L), "mask pass"))) return st;
     if (g_ev_start && g_ev_stop) cudaEventRecord(g_ev_start, L.stream);
     if ((st = lf_cuda(lf_launch_simt_fwd(L, q_s, k_s, v_s, q_g, k_g, v_g, o, lse), "forward")))
       return st;

@@ -165,6 +165,8 @@ struct LfLaunch {
 };
 
 cudaError_t lf_launch_mask_pass(const LfLaunch &L);
+cudaError_t lf_launch_mask_gather(const LfLaunch &L, const void *qg, const void *ks, const void *vs,
+                                  void *qg_c, void *ks_c, void *vs_c, int Ga, int Gka);
 cudaError_t lf_launch_count(const LfLaunch &L, int64_t *counts);
 cudaError_t lf_launch_decode(const LfLaunch &L, const void *q, const void *kc, const void *vc,
                              const int32_t *lengths, void *o, float *lse);

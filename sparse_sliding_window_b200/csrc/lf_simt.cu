@@ -9,21 +9,25 @@
 // (dK, dV); lane l owns head-dim elements 2l and 2l+1, so every K/V/Q row
 // read is one coalesced 128/256-byte access and each score is a warp sum.
 // All sums are float32; outputs are rounded once (RNE) to the call's dtype.
+#include <cooperative_groups.h>
 #include <cub/block/block_scan.cuh>
+
+namespace cg = cooperative_groups;
 
 #include "lf_common.cuh"
 
 // =============================================================== mask pass
 
-// One block per sequence b: compact the global positions (ascending) into
-// gidx[b][0..ng), write the rank array grank[b][p] = #globals before p,
-// count valid tokens, flag bad codes, too many globals and
-// causal+global in the status word.
-__global__ void __launch_bounds__(1024) lf_mask_pass_kernel(LfDev P) {
-  typedef cub::BlockScan<int, 1024> Scan;
-  __shared__ typename Scan::TempStorage tmp;
+// The mask scan of sequence b by one block of 1024 threads: compact the
+// global positions (ascending) into gl_out[0..min(ng, G)), and, when
+// write_tables, write the rank array grank[b][p] = #globals before p, the
+// per-sequence info, and the status flags (bad codes, too many globals,
+// causal + global).  Returns the number of global tokens (all of them).
+typedef cub::BlockScan<int, 1024> LfScan;
+__device__ int lf_mask_scan(const LfDev &P, int b, bool write_tables, int32_t *gl_out,
+                            typename LfScan::TempStorage &tmp) {
   __shared__ int s_valid, s_gmin, s_gmax, s_bad, s_total;
-  const int b = blockIdx.x, tid = threadIdx.x, n = P.n;
+  const int tid = threadIdx.x, n = P.n;
   const int32_t *m = P.mask + (size_t)b * n;
   if (tid == 0) {
     s_valid = 0;
@@ -46,24 +50,23 @@ __global__ void __launch_bounds__(1024) lf_mask_pass_kernel(LfDev P) {
     if (x < 0 || x > 2) bad = 1;
   }
   int off, total;
-  Scan(tmp).ExclusiveSum(c, off, total);
+  LfScan(tmp).ExclusiveSum(c, off, total);
   atomicAdd(&s_valid, v);
   atomicMin(&s_gmin, gmin);
   atomicMax(&s_gmax, gmax);
   if (bad) atomicOr(&s_bad, 1);
   if (tid == 0) s_total = total;
-  int32_t *gl = P.gidx + (size_t)b * P.G;
   int32_t *gr = P.grank + (size_t)b * (n + 1);
   for (int i = s; i < e; i++) {
-    gr[i] = off;  // globals before position i
+    if (write_tables) gr[i] = off;  // globals before position i
     if (m[i] == 2) {
-      if (off < P.G) gl[off] = i;
+      if (off < P.G) gl_out[off] = i;
       off++;
     }
   }
-  if (tid == 1023) gr[n] = total;
+  if (write_tables && tid == 1023) gr[n] = total;
   __syncthreads();
-  if (tid == 0) {
+  if (write_tables && tid == 0) {
     int32_t *bi = P.binfo + (size_t)b * LF_BI_WORDS;
     bi[LF_BI_NG] = min(s_total, P.G);
     bi[LF_BI_NVALID] = s_valid;
@@ -73,10 +76,66 @@ __global__ void __launch_bounds__(1024) lf_mask_pass_kernel(LfDev P) {
     if (s_total > P.G) lf_set_status(P.status, LF_ERR_DEVICE_INPUT, 2000000 + b);
     if (P.causal && s_total > 0) lf_set_status(P.status, LF_ERR_UNSUPPORTED, 3000000 + b);
   }
+  return s_total;
+}
+
+// One block per sequence b: the mask scan and its tables.
+__global__ void __launch_bounds__(1024) lf_mask_pass_kernel(LfDev P) {
+  __shared__ typename LfScan::TempStorage tmp;
+  const int b = blockIdx.x;
+  lf_mask_scan(P, b, true, P.gidx + (size_t)b * P.G, tmp);
 }
 
 cudaError_t lf_launch_mask_pass(const LfLaunch &L) {
   lf_mask_pass_kernel<<<L.dev.B, 1024, 0, L.stream>>>(L.dev);
+  lf_launches_add(1);
+  return cudaGetLastError();
+}
+
+// One block per (b, h): the mask scan of sequence b (block h = 0 also writes
+// its tables and the global list) followed by the compaction of head h's Q_g / K_s / V_s rows of
+// the global tokens (rows past the sequence's global count are zero) -- the
+// mask pass and the gather of the tensor-core forward in one launch.  The
+// global list is kept in shared memory (G entries).
+template <typename T>
+__global__ void __launch_bounds__(1024)
+    lf_mask_gather_kernel(LfDev P, const T *qg, const T *ks, const T *vs, T *qg_c, T *ks_c, T *vs_c,
+                          int Ga, int Gka) {
+  __shared__ typename LfScan::TempStorage tmp;
+  extern __shared__ int32_t s_gl[];
+  const int bh = blockIdx.x, b = bh / P.H;
+  const bool tables = bh % P.H == 0;
+  const int ng = min(lf_mask_scan(P, b, tables, s_gl, tmp), P.G);
+  __syncthreads();
+  if (tables)  // the global list itself, as the mask pass writes it
+    for (int e = threadIdx.x; e < ng; e += blockDim.x) P.gidx[(size_t)b * P.G + e] = s_gl[e];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = warp; e < Gka; e += 32) {
+    uint32_t q = 0, k = 0, v = 0;
+    if (e < ng) {
+      const size_t src = ((size_t)bh * P.n + s_gl[e]) * LF_HD + 2 * lane;
+      q = *reinterpret_cast<const uint32_t *>(qg + src);
+      k = *reinterpret_cast<const uint32_t *>(ks + src);
+      v = *reinterpret_cast<const uint32_t *>(vs + src);
+    }
+    if (e < Ga) *reinterpret_cast<uint32_t *>(qg_c + ((size_t)bh * Ga + e) * LF_HD + 2 * lane) = q;
+    *reinterpret_cast<uint32_t *>(ks_c + ((size_t)bh * Gka + e) * LF_HD + 2 * lane) = k;
+    *reinterpret_cast<uint32_t *>(vs_c + ((size_t)bh * Gka + e) * LF_HD + 2 * lane) = v;
+  }
+}
+
+cudaError_t lf_launch_mask_gather(const LfLaunch &L, const void *qg, const void *ks, const void *vs,
+                                  void *qg_c, void *ks_c, void *vs_c, int Ga, int Gka) {
+  const unsigned grid = (unsigned)(L.dev.B * L.dev.H);
+  const size_t sm = (size_t)L.dev.G * sizeof(int32_t);
+  if (L.dtype == LF_F16)
+    lf_mask_gather_kernel<__half><<<grid, 1024, sm, L.stream>>>(
+        L.dev, (const __half *)qg, (const __half *)ks, (const __half *)vs, (__half *)qg_c,
+        (__half *)ks_c, (__half *)vs_c, Ga, Gka);
+  else
+    lf_mask_gather_kernel<__nv_bfloat16><<<grid, 1024, sm, L.stream>>>(
+        L.dev, (const __nv_bfloat16 *)qg, (const __nv_bfloat16 *)ks, (const __nv_bfloat16 *)vs,
+        (__nv_bfloat16 *)qg_c, (__nv_bfloat16 *)ks_c, (__nv_bfloat16 *)vs_c, Ga, Gka);
   lf_launches_add(1);
   return cudaGetLastError();
 }
@@ -559,38 +618,44 @@ cudaError_t lf_launch_bwd_delta_dkvg(const LfLaunch &L, const void *o, const voi
 
 // ============================================================ decode step
 
-// One block of 8 warps per (b, h): warp w takes the window offsets
-// k = w*32*chunks ... (one key per lane, batches of 32), then the warps merge
-// their (max, sum, partial output) in shared memory.
+// A cluster of LF_DEC_CL CTAs of 4 warps per (b, h): the window offsets go
+// in batches of 32 (one key per lane, as in the CUDA-core forward), warp w of
+// CTA c taking batches c*4 + w, + 4*LF_DEC_CL, ...  Each CTA merges its
+// warps' (max, sum, partial output) in shared memory and writes the result
+// into CTA 0's shared memory (distributed shared memory); CTA 0 merges the
+// cluster's partials and writes o and lse.  One window of r + 1 keys is a
+// few hundred KB at most, so the step is latency-bound: spreading it over
+// 32 warps on 8 SMs keeps each warp at one or two batches.
+#define LF_DEC_CL 8
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __cluster_dims__(LF_DEC_CL, 1, 1) __launch_bounds__(128)
     lf_decode_kernel(LfDev P, const T *q, const T *kc, const T *vc, const int32_t *lengths, T *o,
                      float *lse) {
-  __shared__ float s_m[8], s_l[8], s_acc[8][LF_HD];
-  const int bh = blockIdx.x, h = bh % P.H, b = bh / P.H, d = P.dil[h], n = P.n;
+  __shared__ float s_m[4], s_l[4], s_acc[4][LF_HD];
+  __shared__ float c_m[LF_DEC_CL], c_l[LF_DEC_CL], c_acc[LF_DEC_CL][LF_HD];  // used in CTA 0
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = (int)cluster.block_rank();
+  const int bh = blockIdx.x / LF_DEC_CL, h = bh % P.H, b = bh / P.H, d = P.dil[h], n = P.n;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = lengths[b];
   const size_t obase = (size_t)bh * LF_HD;
-  if (L < 1 || L > n) {
-    if (warp == 0) {
-      LfIo<T>::st2(o + obase + 2 * lane, 0.f, 0.f);
-      if (lse && lane == 0) lse[bh] = -INFINITY;
-    }
-    return;
-  }
-  const int t = L - 1;
-  const int kmax = min(P.r, t / d);  // keys j = t - k*d >= 0
-  const size_t base = (size_t)bh * n * LF_HD;
+  const bool valid = L >= 1 && L <= n;
+  cluster.sync();  // every CTA of the cluster runs before any remote access
   LfRowAcc<T> st;
-  lf_load_row64<T>(q + obase, st.q);
-#pragma unroll
-  for (int c = 0; c < 64; c++) st.q[c] *= P.scale_log2;
   st.mx = -INFINITY;
   st.l = st.a0 = st.a1 = 0.f;
-  st.self = t;
-  for (int k0 = warp * 32; k0 <= kmax; k0 += 8 * 32) {
-    const int k = k0 + lane;
-    st.batch(kc, vc, base, t - k * d, k <= kmax, lane);
+  if (valid) {
+    const int t = L - 1;
+    const int kmax = min(P.r, t / d);  // keys j = t - k*d >= 0
+    const size_t base = (size_t)bh * n * LF_HD;
+    lf_load_row64<T>(q + obase, st.q);
+#pragma unroll
+    for (int c = 0; c < 64; c++) st.q[c] *= P.scale_log2;
+    st.self = t;
+    for (int k0 = (crank * 4 + warp) * 32; k0 <= kmax; k0 += 4 * LF_DEC_CL * 32) {
+      const int k = k0 + lane;
+      st.batch(kc, vc, base, t - k * d, k <= kmax, lane);
+    }
   }
   if (lane == 0) {
     s_m[warp] = st.mx;
@@ -600,17 +665,46 @@ __global__ void __launch_bounds__(256)
   s_acc[warp][2 * lane + 1] = st.a1;
   __syncthreads();
   if (warp == 0) {
+    // this CTA's partial, into slot crank of CTA 0
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < 8; w++) M = fmaxf(M, s_m[w]);
+    for (int w = 0; w < 4; w++) M = fmaxf(M, s_m[w]);
     float Ls = 0.f, a0 = 0.f, a1 = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; w++) {
+    for (int w = 0; w < 4; w++) {
       if (s_m[w] == -INFINITY) continue;
       const float f = exp2f(s_m[w] - M);
       Ls += s_l[w] * f;
       a0 += s_acc[w][2 * lane] * f;
       a1 += s_acc[w][2 * lane + 1] * f;
+    }
+    float *rm = cluster.map_shared_rank(c_m, 0), *rl = cluster.map_shared_rank(c_l, 0);
+    float *racc = cluster.map_shared_rank(&c_acc[0][0], 0);
+    if (lane == 0) {
+      rm[crank] = M;
+      rl[crank] = Ls;
+    }
+    racc[crank * LF_HD + 2 * lane] = a0;
+    racc[crank * LF_HD + 2 * lane + 1] = a1;
+  }
+  cluster.sync();  // partials in CTA 0
+  if (crank == 0 && warp == 0) {
+    if (!valid) {
+      LfIo<T>::st2(o + obase + 2 * lane, 0.f, 0.f);
+      if (lse && lane == 0) lse[bh] = -INFINITY;
+      return;
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < LF_DEC_CL; c++) M = fmaxf(M, c_m[c]);
+    float Ls = 0.f, a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < LF_DEC_CL; c++) {
+      if (c_m[c] == -INFINITY) continue;
+      const float f = exp2f(c_m[c] - M);
+      Ls += c_l[c] * f;
+      a0 += c_acc[c][2 * lane] * f;
+      a1 += c_acc[c][2 * lane + 1] * f;
     }
     LfIo<T>::st2(o + obase + 2 * lane, a0 / Ls, a1 / Ls);
     if (lse && lane == 0) lse[bh] = (M + log2f(Ls)) * LF_LN2;
@@ -619,19 +713,19 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t lf_launch_decode(const LfLaunch &L, const void *q, const void *kc, const void *vc,
                              const int32_t *lengths, void *o, float *lse) {
-  const unsigned grid = (unsigned)(L.dev.B * L.dev.H);
+  const unsigned grid = (unsigned)(L.dev.B * L.dev.H * LF_DEC_CL);
   switch (L.dtype) {
     case LF_F32:
-      lf_decode_kernel<float><<<grid, 256, 0, L.stream>>>(L.dev, (const float *)q, (const float *)kc,
+      lf_decode_kernel<float><<<grid, 128, 0, L.stream>>>(L.dev, (const float *)q, (const float *)kc,
                                                           (const float *)vc, lengths, (float *)o, lse);
       break;
     case LF_BF16:
-      lf_decode_kernel<__nv_bfloat16><<<grid, 256, 0, L.stream>>>(
+      lf_decode_kernel<__nv_bfloat16><<<grid, 128, 0, L.stream>>>(
           L.dev, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)kc, (const __nv_bfloat16 *)vc,
           lengths, (__nv_bfloat16 *)o, lse);
       break;
     default:
-      lf_decode_kernel<__half><<<grid, 256, 0, L.stream>>>(L.dev, (const __half *)q, (const __half *)kc,
+      lf_decode_kernel<__half><<<grid, 128, 0, L.stream>>>(L.dev, (const __half *)q, (const __half *)kc,
                                                            (const __half *)vc, lengths, (__half *)o, lse);
   }
   lf_launches_add(1);

@@ -856,12 +856,19 @@ int lf_tc_fwd(const LfLaunch &L, const LfTcArgs &a, char *err, size_t errlen) {
     P.part_acc = (float *)(L.ws_base + L.ws.part_acc);
     P.part_ml = (float2 *)(L.ws_base + L.ws.part_ml);
     (void)eb;
-    if (G > 0) {
-      cudaError_t e = lf_launch_gather(L, a.qg, a.ks, a.vs, qg_c, ks_c, vs_c, Ga, Gka);
-      if (e != cudaSuccess) {
-        snprintf(err, errlen, "gather launch: %s", cudaGetErrorString(e));
-        return LF_ERR_CUDA;
-      }
+    // the mask pass (global list, rank array, sequence info, input checks),
+    // fused with the compaction of the global tokens' rows when the list
+    // fits in shared memory
+    cudaError_t e;
+    if (G > 0 && G <= 8192) {  // list in shared memory: 32 KB at most
+      e = lf_launch_mask_gather(L, a.qg, a.ks, a.vs, qg_c, ks_c, vs_c, Ga, Gka);
+    } else {
+      e = lf_launch_mask_pass(L);
+      if (e == cudaSuccess && G > 0) e = lf_launch_gather(L, a.qg, a.ks, a.vs, qg_c, ks_c, vs_c, Ga, Gka);
+    }
+    if (e != cudaSuccess) {
+      snprintf(err, errlen, "mask pass / gather launch: %s", cudaGetErrorString(e));
+      return LF_ERR_CUDA;
     }
   }
   {

@@ -82,6 +82,7 @@ __device__ int lf_mask_scan(const LfDev &P, int b, bool write_tables, int32_t *g
 // One block per sequence b: the mask scan and its tables.
 __global__ void __launch_bounds__(1024) lf_mask_pass_kernel(LfDev P) {
   __shared__ typename LfScan::TempStorage tmp;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = blockIdx.x;
   lf_mask_scan(P, b, true, P.gidx + (size_t)b * P.G, tmp);
 }
@@ -103,6 +104,8 @@ __global__ void __launch_bounds__(1024)
                           int Ga, int Gka) {
   __shared__ typename LfScan::TempStorage tmp;
   extern __shared__ int32_t s_gl[];
+  // the forward kernel launched after this one may start its set-up now
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int bh = blockIdx.x, b = bh / P.H;
   const bool tables = bh % P.H == 0;
   const int ng = min(lf_mask_scan(P, b, tables, s_gl, tmp), P.G);

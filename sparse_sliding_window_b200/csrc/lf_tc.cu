@@ -292,6 +292,11 @@ __global__ void __launch_bounds__(LF_TC_THREADS, 1)
   __syncthreads();
   lf_tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // launched as a programmatic dependent of the mask pass: the set-up above
+  // overlaps its tail; its tables (global list, ranks, compacted rows) are
+  // read only after it has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the combine kernel
 
   // consumers take the stream's items from its two slots in order; -1 ends
   auto take_item = [&](int k, int &idx) -> bool {
@@ -706,6 +711,7 @@ __global__ void __launch_bounds__(256)
 template <typename T>
 __global__ void __launch_bounds__(256)
     lf_combine_kernel(LfDev D, const float *part_acc, const float2 *part_ml, T *o, float *lse) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the partials of the forward kernel
   const int lane = threadIdx.x & 31;
   const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (w >= (long long)D.B * D.H * D.G) return;
@@ -781,6 +787,29 @@ cudaError_t lf_launch_gather(const LfLaunch &L, const void *qg, const void *ks, 
         (__nv_bfloat16 *)qg_c, (__nv_bfloat16 *)ks_c, (__nv_bfloat16 *)vs_c, Ga, Gka);
   lf_launches_add(1);
   return cudaGetLastError();
+}
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on the stream finishes, and waits for it (griddepcontrol)
+// before reading its results.
+static cudaError_t lf_launch_pdl_args(const void *fn, unsigned grid, unsigned block, size_t smem,
+                                      cudaStream_t stream, void **args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+static cudaError_t lf_launch_pdl(const void *fn, unsigned grid, unsigned block, size_t smem,
+                                 cudaStream_t stream, LfTcParams *P) {
+  void *args[] = {(void *)P};
+  return lf_launch_pdl_args(fn, grid, block, smem, stream, args);
 }
 
 static bool lf_tc_attr_done[2] = {false, false};
@@ -892,10 +921,10 @@ int lf_tc_fwd(const LfLaunch &L, const LfTcArgs &a, char *err, size_t errlen) {
     const unsigned grid = (unsigned)std::min<long long>(items, nsm);  // persistent: one CTA per SM
     P.sched_cta = items <= 4LL * grid ? 1 : 0;
     if (a.ev_start && a.ev_stop) cudaEventRecord(a.ev_start, L.stream);
-    kern<<<grid, LF_TC_THREADS, LF_SMEM_BYTES, L.stream>>>(P);
+    cudaError_t le = lf_launch_pdl((const void *)kern, grid, LF_TC_THREADS, LF_SMEM_BYTES, L.stream, &P);
     lf_launches_add(1);
     if (a.ev_start && a.ev_stop) cudaEventRecord(a.ev_stop, L.stream);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = le != cudaSuccess ? le : cudaGetLastError();
     if (e != cudaSuccess) {
       snprintf(err, errlen, "tensor-core forward launch: %s", cudaGetErrorString(e));
       return LF_ERR_CUDA;
@@ -904,14 +933,20 @@ int lf_tc_fwd(const LfLaunch &L, const LfTcArgs &a, char *err, size_t errlen) {
   if (D.G > 0) {
     const long long rows = (long long)D.B * D.H * D.G;
     const unsigned grid = (unsigned)((rows + 7) / 8);
-    if (f16)
-      lf_combine_kernel<__half><<<grid, 256, 0, L.stream>>>(
-          D, (const float *)P.part_acc, (const float2 *)P.part_ml, (__half *)a.o, a.lse);
-    else
-      lf_combine_kernel<__nv_bfloat16><<<grid, 256, 0, L.stream>>>(
-          D, (const float *)P.part_acc, (const float2 *)P.part_ml, (__nv_bfloat16 *)a.o, a.lse);
+    const float *pacc = (const float *)P.part_acc;
+    const float2 *pml = (const float2 *)P.part_ml;
+    cudaError_t le;
+    if (f16) {
+      __half *o = (__half *)a.o;
+      void *args[] = {(void *)&D, (void *)&pacc, (void *)&pml, (void *)&o, (void *)&a.lse};
+      le = lf_launch_pdl_args((const void *)lf_combine_kernel<__half>, grid, 256, 0, L.stream, args);
+    } else {
+      __nv_bfloat16 *o = (__nv_bfloat16 *)a.o;
+      void *args[] = {(void *)&D, (void *)&pacc, (void *)&pml, (void *)&o, (void *)&a.lse};
+      le = lf_launch_pdl_args((const void *)lf_combine_kernel<__nv_bfloat16>, grid, 256, 0, L.stream, args);
+    }
     lf_launches_add(1);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = le != cudaSuccess ? le : cudaGetLastError();
     if (e != cudaSuccess) {
       snprintf(err, errlen, "combine launch: %s", cudaGetErrorString(e));
       return LF_ERR_CUDA;

@@ -1,7 +1,7 @@
 // lf_tc.cu -- tensor-core (tcgen05 / TMEM / TMA) forward of Longformer
 // attention for sm_100a, bf16 or f16 inputs, fp32 accumulation.
 //
-// One kernel runs two kinds of work items, one item per CTA:
+// One kernel runs two kinds of work items:
 //
 //  * BAND items: 128 query rows t0..t0+127 of one (b, h, residue rho).  A
 //    head with dilation d is split into its d residue sub-sequences
@@ -22,27 +22,27 @@
 //    全局注意力).  Each writes an unnormalised partial (acc, max, sum) that
 //    lf_combine_kernel merges (split-KV).
 //
-// Persistent: one CTA of 320 threads per SM walks the work items
-// blockIdx.x, blockIdx.x + gridDim.x, ...  Warp 8 issues TMA loads (Q per
-// item into one of two buffers, K/V tiles into a 5-stage ring that runs
-// ahead into the next item), warp 9 owns all 512 TMEM columns and issues
-// the tcgen05.mma instructions, and two softmax
-// groups of four warps (warps 0-3, 4-7; one TMEM lane = one query row per
-// thread) take the key tiles of an item in turn: group 0 tiles 0, 2, 4, ..., group 1 tiles 1, 3, 5, ...  Each group
-// has its own S tile, O accumulator and P tile in TMEM
-// (S_g = [128g, 128g+128), O_g = [256+64g, +64), P_g = [384+64g, +64)), so
-// one group's softmax overlaps the tensor-core work of the other's.
-// Per tile t of group g:
-//             MMA  S_g = Q K_t^T                       -> commit s_full(g)
-//             SMX  P_g = exp2(S*scale*log2e - m) against the running max m
-//                  (redone with a new m, O_g rescaled, when a row max grew
-//                  by more than 2^8), row sum
-//                                                      -> arrive p_full(g)
-//             MMA  S_g = Q K_{t+2}^T  (next tile of the group) -> s_full(g)
-//             MMA  O_g += P_g V_t (A operand from TMEM) -> kv_empty, pv_done(g)
-// At the end of an item the two groups merge their (max, sum, O) on chip
-// and write O and the log-normaliser, so the n x w score band never leaves
-// the SM.
+// Persistent: one CTA of 384 threads per SM runs two independent streams.
+// Stream g has its own producer warp (8 + 2g: takes the next work item and
+// issues its TMA loads -- Q into the stream's buffer, K/V tiles into its
+// 3-stage ring), MMA warp (9 + 2g: issues the tcgen05.mma phases from one
+// elected lane), four softmax warps (4g .. 4g+3: one TMEM lane = one query
+// row per thread) and 256 TMEM columns (S tile, O accumulator, P tile).  A
+// stream processes whole items, so nothing is merged between streams; while
+// one stream waits for its next S tile the other keeps the SM's exp unit
+// busy.  Items come largest first, from the CTA's own list when there are
+// few per SM and from one grid-wide counter otherwise.
+// Per tile t of an item:
+//             SMX  attend mask of the row for tile t (while S is in flight)
+//             MMA  S = Q K_t^T                            -> commit s_full
+//             SMX  P = exp2(S*scale*log2e - m) against the row's running
+//                  reference m (the tile is redone with its own max, O
+//                  rescaled, when the row sum leaves the P format's safe
+//                  range), row sum                       -> arrive p_full
+//             MMA  S = Q K_{t+1}^T                        -> commit s_full
+//             MMA  O += P V_t (A operand from TMEM)       -> kv_empty, pv_done
+// After the item's last tile the softmax warps write O / l and the
+// log-normaliser, so the n x w score band never leaves the SM.
 //
 // Every wait is bounded: after LF_WAIT_NS without progress the waiting
 // thread records LF_ERR_DEVICE_TIMEOUT in the status word, raises the CTA's

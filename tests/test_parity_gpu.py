@@ -87,6 +87,26 @@ def _setup(name, dtype, kernel, seed=11, backward=False):
     return c, wl, inp, att
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_forward_default_max_global_long_sequence(dtype):
+    """max_global left at its default (-1: room for n global rows) on a
+    sequence longer than 8192: the global list no longer fits the fused mask
+    pass + gather kernel, so the separate mask pass and gather kernels run."""
+    n = 8500
+    m = _mask(1, n, globals_=[[0, 4000, n - 1]])
+    wl = synth.custom("long_default_g", 1, 1, n, 32, [1], False, dtype, m, seed=23)
+    inp = synth.inputs_for(wl)
+    att = L.LongformerAttention(1, 1, n, 32, [1], False, dtype=dtype, kernel=L.LF_KERNEL_TC)
+    g = U.gpu_inputs(inp, dtype)
+    o, lse = att.fwd(g["qs"], g["ks"], g["vs"], g["qg"], g["kg"], g["vg"], g["mask"])
+    att.status()
+    f = U.f64_inputs(inp, dtype)
+    ro, rl = oracle.fwd(32, [1], False, U.scale_of(wl), inp["mask"], f["qs"], f["ks"], f["vs"],
+                        f["qg"], f["kg"], f["vg"])
+    U.compare("long_default_g/o", U.to_f64(o), ro, dtype)
+    U.compare_lse(U.to_f64(lse), rl, dtype)
+
+
 @pytest.mark.parametrize("dtype,kernel", KERNELS)
 @pytest.mark.parametrize("name", sorted(CASES))
 def test_forward_parity(name, dtype, kernel):

@@ -522,36 +522,53 @@ template <typename T>
 __global__ void __launch_bounds__(256)
     lf_bwd_dkv_g_kernel(LfDev P, const T *qg, const T *kg, const T *vg, const float *lse,
                         const T *dO, const float *delta, T *dkg, T *dvg) {
+  // one warp per 8 consecutive keys j of one (b, h); the global rows' Q_g /
+  // dO rows are shared by the 8 keys, the 8 keys' loads are issued together
   const int lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int n = P.n;
-  if (row >= (long long)P.B * P.H * n) return;
-  const int j = (int)(row % n);
-  const int bh = (int)(row / n), b = bh / P.H;
+  const int n = P.n, nb = (n + 7) / 8;
+  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (w >= (long long)P.B * P.H * nb) return;
+  const int jb = (int)(w % nb) * 8;
+  const int bh = (int)(w / nb), b = bh / P.H;
   const int32_t *m = P.mask + (size_t)b * n;
   const size_t base = (size_t)bh * n * LF_HD + 2 * lane;
-  const size_t joff = base + (size_t)j * LF_HD;
-  float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
-  if (m[j] != 0) {
-    float2 kk = LfIo<T>::ld2(kg + joff), vv = LfIo<T>::ld2(vg + joff);
-    const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
-    const int32_t *gl = P.gidx + (size_t)b * P.G;
-    for (int t = 0; t < ng; t++) {
-      int i = gl[t];
-      size_t ioff = base + (size_t)i * LF_HD;
-      size_t ir = (size_t)bh * n + i;
-      float2 q = LfIo<T>::ld2(qg + ioff), g = LfIo<T>::ld2(dO + ioff);
-      float2 sd = lf_warp_sum2(q.x * kk.x + q.y * kk.y, g.x * vv.x + g.y * vv.y);
-      float pr = exp2f(sd.x * P.scale_log2 - lse[ir] * LF_LOG2E);
-      float ds = pr * (sd.y - delta[ir]) * P.scale;
-      k0 += ds * q.x;
-      k1 += ds * q.y;
-      v0 += pr * g.x;
-      v1 += pr * g.y;
+  float2 kk[8], vv[8];
+  float k0[8], k1[8], v0[8], v1[8];
+  bool on[8];
+#pragma unroll
+  for (int u = 0; u < 8; u++) {
+    const int j = min(jb + u, n - 1);
+    kk[u] = LfIo<T>::ld2(kg + base + (size_t)j * LF_HD);
+    vv[u] = LfIo<T>::ld2(vg + base + (size_t)j * LF_HD);
+    on[u] = jb + u < n && m[j] != 0;
+    k0[u] = k1[u] = v0[u] = v1[u] = 0.f;
+  }
+  const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
+  const int32_t *gl = P.gidx + (size_t)b * P.G;
+  for (int t = 0; t < ng; t++) {
+    const int i = gl[t];
+    const size_t ioff = base + (size_t)i * LF_HD, ir = (size_t)bh * n + i;
+    const float2 q = LfIo<T>::ld2(qg + ioff), g = LfIo<T>::ld2(dO + ioff);
+    const float L2 = lse[ir] * LF_LOG2E, Dg = delta[ir];
+#pragma unroll
+    for (int u = 0; u < 8; u++) {
+      if (!on[u]) continue;
+      const float2 sd = lf_warp_sum2(q.x * kk[u].x + q.y * kk[u].y, g.x * vv[u].x + g.y * vv[u].y);
+      const float pr = exp2f(sd.x * P.scale_log2 - L2);
+      const float ds = pr * (sd.y - Dg) * P.scale;
+      k0[u] += ds * q.x;
+      k1[u] += ds * q.y;
+      v0[u] += pr * g.x;
+      v1[u] += pr * g.y;
     }
   }
-  LfIo<T>::st2(dkg + joff, k0, k1);
-  LfIo<T>::st2(dvg + joff, v0, v1);
+#pragma unroll
+  for (int u = 0; u < 8; u++) {
+    if (jb + u >= n) break;
+    const size_t joff = base + (size_t)(jb + u) * LF_HD;
+    LfIo<T>::st2(dkg + joff, k0[u], k1[u]);
+    LfIo<T>::st2(dvg + joff, v0[u], v1[u]);
+  }
 }
 
 template <typename T>
@@ -569,7 +586,8 @@ static cudaError_t lf_simt_bwd_t(const LfLaunch &L, const void *qs, const void *
   lf_bwd_dkv_s_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)qs, (const T *)ks,
                                                      (const T *)vs, lse, (const T *)dO, delta,
                                                      (T *)dks, (T *)dvs);
-  lf_bwd_dkv_g_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)qg, (const T *)kg,
+  const long long w8 = (long long)L.dev.B * L.dev.H * ((L.dev.n + 7) / 8);  // 8 keys per warp
+  lf_bwd_dkv_g_kernel<T><<<(unsigned)((w8 + 7) / 8), 256, 0, L.stream>>>(L.dev, (const T *)qg, (const T *)kg,
                                                      (const T *)vg, lse, (const T *)dO, delta,
                                                      (T *)dkg, (T *)dvg);
   lf_launches_add(4);
@@ -602,7 +620,8 @@ static cudaError_t lf_bwd_delta_dkvg_t(const LfLaunch &L, const void *o, const v
   long long rows = (long long)L.dev.B * L.dev.H * L.dev.n;
   unsigned grid = (unsigned)((rows + 7) / 8);
   lf_bwd_delta_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)o, (const T *)dO, delta);
-  lf_bwd_dkv_g_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)qg, (const T *)kg,
+  const long long w8 = (long long)L.dev.B * L.dev.H * ((L.dev.n + 7) / 8);
+  lf_bwd_dkv_g_kernel<T><<<(unsigned)((w8 + 7) / 8), 256, 0, L.stream>>>(L.dev, (const T *)qg, (const T *)kg,
                                                      (const T *)vg, lse, (const T *)dO, delta,
                                                      (T *)dkg, (T *)dvg);
   lf_launches_add(2);

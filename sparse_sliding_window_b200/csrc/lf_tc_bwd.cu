@@ -478,18 +478,34 @@ __global__ void __launch_bounds__(256)
     const size_t base = (size_t)bh * n * LF_HD + 2 * lane;
     const float2 kk = LfIo<T>::ld2(ks + base + (size_t)g * LF_HD);
     const float2 vv = LfIo<T>::ld2(vs + base + (size_t)g * LF_HD);
-    const int i1 = min(n, (c + 1) * LF_BW_ROWS_PER_CHUNK);
-    for (int i = c * LF_BW_ROWS_PER_CHUNK; i < i1; i++) {
-      if (m[i] != 1 || lf_in_window(i, g, P.r, d, P.causal)) continue;
-      const size_t ioff = base + (size_t)i * LF_HD, ir = (size_t)bh * n + i;
-      const float2 q = LfIo<T>::ld2(qs + ioff), go = LfIo<T>::ld2(dO + ioff);
-      const float2 sd = lf_warp_sum2(q.x * kk.x + q.y * kk.y, go.x * vv.x + go.y * vv.y);
-      const float pr = exp2f(sd.x * P.scale_log2 - lse[ir] * LF_LOG2E);
-      const float ds = pr * (sd.y - delta[ir]) * P.scale;
-      k0 += ds * q.x;
-      k1 += ds * q.y;
-      v0 += pr * go.x;
-      v1 += pr * go.y;
+    const int i0 = c * LF_BW_ROWS_PER_CHUNK, i1 = min(n, i0 + LF_BW_ROWS_PER_CHUNK);
+    // rows in batches of 8: every load of a batch is issued before the first
+    // use (a row outside the chunk reads row i1 - 1 and is skipped); the sums
+    // run in row order as before
+    for (int ib = i0; ib < i1; ib += 8) {
+      float2 q[8], go[8];
+      float ls[8], dl[8];
+#pragma unroll
+      for (int u = 0; u < 8; u++) {
+        const int i = min(ib + u, i1 - 1);
+        const size_t ioff = base + (size_t)i * LF_HD, ir = (size_t)bh * n + i;
+        q[u] = LfIo<T>::ld2(qs + ioff);
+        go[u] = LfIo<T>::ld2(dO + ioff);
+        ls[u] = lse[ir];
+        dl[u] = delta[ir];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; u++) {
+        const int i = ib + u;
+        if (i >= i1 || m[i] != 1 || lf_in_window(i, g, P.r, d, P.causal)) continue;
+        const float2 sd = lf_warp_sum2(q[u].x * kk.x + q[u].y * kk.y, go[u].x * vv.x + go[u].y * vv.y);
+        const float pr = exp2f(sd.x * P.scale_log2 - ls[u] * LF_LOG2E);
+        const float ds = pr * (sd.y - dl[u]) * P.scale;
+        k0 += ds * q[u].x;
+        k1 += ds * q[u].y;
+        v0 += pr * go[u].x;
+        v1 += pr * go[u].y;
+      }
     }
   }
   float *dst = part + ((size_t)be * nch + c) * 2 * LF_HD + 2 * lane;
@@ -549,16 +565,26 @@ __global__ void __launch_bounds__(256)
     const float2 q = LfIo<T>::ld2(qg + base + (size_t)g * LF_HD);
     const float2 go = LfIo<T>::ld2(dO + base + (size_t)g * LF_HD);
     const float L2 = lse[gr] * LF_LOG2E, Dg = delta[gr];
-    const int j1 = min(n, (c + 1) * LF_BW_ROWS_PER_CHUNK);
-    for (int j = c * LF_BW_ROWS_PER_CHUNK; j < j1; j++) {
-      if (m[j] == 0) continue;
-      const size_t joff = base + (size_t)j * LF_HD;
-      const float2 k = LfIo<T>::ld2(kg + joff), v = LfIo<T>::ld2(vg + joff);
-      const float2 sd = lf_warp_sum2(q.x * k.x + q.y * k.y, go.x * v.x + go.y * v.y);
-      const float pr = exp2f(sd.x * P.scale_log2 - L2);
-      const float ds = pr * (sd.y - Dg) * P.scale;
-      a0 += ds * k.x;
-      a1 += ds * k.y;
+    const int j0 = c * LF_BW_ROWS_PER_CHUNK, j1 = min(n, j0 + LF_BW_ROWS_PER_CHUNK);
+    // keys in batches of 8, every load issued before the first use; sums in key order
+    for (int jb = j0; jb < j1; jb += 8) {
+      float2 k[8], v[8];
+#pragma unroll
+      for (int u = 0; u < 8; u++) {
+        const size_t joff = base + (size_t)min(jb + u, j1 - 1) * LF_HD;
+        k[u] = LfIo<T>::ld2(kg + joff);
+        v[u] = LfIo<T>::ld2(vg + joff);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; u++) {
+        const int j = jb + u;
+        if (j >= j1 || m[j] == 0) continue;
+        const float2 sd = lf_warp_sum2(q.x * k[u].x + q.y * k[u].y, go.x * v[u].x + go.y * v[u].y);
+        const float pr = exp2f(sd.x * P.scale_log2 - L2);
+        const float ds = pr * (sd.y - Dg) * P.scale;
+        a0 += ds * k[u].x;
+        a1 += ds * k[u].y;
+      }
     }
   }
   *reinterpret_cast<float2 *>(part + ((size_t)be * nch + c) * LF_HD + 2 * lane) = make_float2(a0, a1);

@@ -56,6 +56,8 @@ def _cases():
     C["window_ge_n"] = dict(B=1, H=2, n=200, r=300, dil=[1, 3], causal=False,
                             mask=_mask(1, 200, globals_=[[7]]))
     C["n1"] = dict(B=1, H=1, n=1, r=4, dil=[1], causal=False, mask=_mask(1, 1))
+    # a causal window wider than the sequence: full causal (decoder) self-attention
+    C["causal_dense"] = dict(B=1, H=2, n=600, r=1000, dil=[1, 1], causal=True, mask=_mask(1, 600))
     # large scores (inputs N(0, 3^2) / N(0, 4^2)): row sums leave the range the
     # running reference allows, so the tensor-core softmax redoes tiles with
     # the row's tile max (overflow side) and, with two keys per row, with

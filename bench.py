@@ -138,7 +138,7 @@ def job_throughput(units_per_rank: int, world: int, ms_per_step: float) -> float
 # DRAM traffic of the main forward kernel per launch, from the ncu captures
 # summarised under profiles/; reported only while the kernel sources are the
 # ones that were profiled (their sha256 prefix), else null.
-PROFILED_TRAFFIC = {"base_bf16": {"bytes": 31917824, "sha": "10cd39424e4783f8"}}
+PROFILED_TRAFFIC = {"base_bf16": {"bytes": 31917824, "sha": "ae00b96c2645de78"}}
 
 
 def kernel_traffic(workload: str):

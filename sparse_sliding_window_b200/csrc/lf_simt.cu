@@ -655,6 +655,8 @@ __global__ void __cluster_dims__(LF_DEC_CL, 1, 1) __launch_bounds__(128)
                      float *lse) {
   __shared__ float s_m[4], s_l[4], s_acc[4][LF_HD];
   __shared__ float c_m[LF_DEC_CL], c_l[LF_DEC_CL], c_acc[LF_DEC_CL][LF_HD];  // used in CTA 0
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the previous kernel's writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = (int)cluster.block_rank();
   const int bh = blockIdx.x / LF_DEC_CL, h = bh % P.H, b = bh / P.H, d = P.dil[h], n = P.n;
@@ -733,23 +735,33 @@ __global__ void __cluster_dims__(LF_DEC_CL, 1, 1) __launch_bounds__(128)
   }
 }
 
+template <typename T>
+static cudaError_t lf_launch_decode_t(const LfLaunch &L, const void *q, const void *kc,
+                                      const void *vc, const int32_t *lengths, void *o, float *lse) {
+  // programmatic dependent launch: a step's launch overlaps the previous
+  // kernel on the stream (the kernel waits for it before reading anything)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(L.dev.B * L.dev.H * LF_DEC_CL));
+  cfg.blockDim = dim3(128);
+  cfg.stream = L.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, lf_decode_kernel<T>, L.dev, (const T *)q, (const T *)kc,
+                            (const T *)vc, lengths, (T *)o, lse);
+}
+
 cudaError_t lf_launch_decode(const LfLaunch &L, const void *q, const void *kc, const void *vc,
                              const int32_t *lengths, void *o, float *lse) {
-  const unsigned grid = (unsigned)(L.dev.B * L.dev.H * LF_DEC_CL);
+  cudaError_t e;
   switch (L.dtype) {
-    case LF_F32:
-      lf_decode_kernel<float><<<grid, 128, 0, L.stream>>>(L.dev, (const float *)q, (const float *)kc,
-                                                          (const float *)vc, lengths, (float *)o, lse);
-      break;
-    case LF_BF16:
-      lf_decode_kernel<__nv_bfloat16><<<grid, 128, 0, L.stream>>>(
-          L.dev, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)kc, (const __nv_bfloat16 *)vc,
-          lengths, (__nv_bfloat16 *)o, lse);
-      break;
-    default:
-      lf_decode_kernel<__half><<<grid, 128, 0, L.stream>>>(L.dev, (const __half *)q, (const __half *)kc,
-                                                           (const __half *)vc, lengths, (__half *)o, lse);
+    case LF_F32: e = lf_launch_decode_t<float>(L, q, kc, vc, lengths, o, lse); break;
+    case LF_BF16: e = lf_launch_decode_t<__nv_bfloat16>(L, q, kc, vc, lengths, o, lse); break;
+    default: e = lf_launch_decode_t<__half>(L, q, kc, vc, lengths, o, lse);
   }
+  if (e != cudaSuccess) return e;
   lf_launches_add(1);
   return cudaGetLastError();
 }

@@ -60,3 +60,18 @@ def test_batched_workload_structure():
         assert np.all(m[b, L:] == 0)  # padding tail
         g = np.flatnonzero(m[b] == 2)
         assert g[0] == 0 and len(g) == 17 and g.max() < L  # token 0 + 16 distinct in [1, L)
+
+
+def test_algorithmic_bytes_of_base_workload():
+    """The roofline denominator of the base workload, counted by hand: Q_s,
+    K_s, V_s read and O written for 12 x 4096 rows of 128 bytes, Q_g at the
+    65 global rows of each head, K_g and V_g in full, the int32 mask and the
+    fp32 log-normaliser."""
+    sys.path.insert(0, ROOT)
+    import bench
+    wl = synth.WORKLOADS["base_bf16"]
+    mask = synth.make_inputs(wl, with_do=False)["mask"]
+    rows = 12 * 4096
+    expect = 4 * rows * 128 + 12 * 65 * 128 + 2 * rows * 128 + 4096 * 4 + rows * 4
+    assert expect == 38061568
+    assert bench.algorithmic_bytes(wl, mask) == expect

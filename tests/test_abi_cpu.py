@@ -80,3 +80,19 @@ def test_host_validation_without_gpu(lib):
     assert rc == L.LF_ERR_INVALID and b"lse" in lib.lf_attn_last_error()
     # NULL params
     assert lib.lf_attn_count_pairs(None, vp(a16), vp(a16), vp(a16), 4096, None) == L.LF_ERR_INVALID
+
+
+def test_decode_host_validation_without_gpu(lib):
+    """The decode entry refuses a non-causal window and bad pointers on the
+    host, before any launch."""
+    buf = (ctypes.c_char * 4096)()
+    a16 = (ctypes.addressof(buf) + 255) & ~255
+    vp = ctypes.c_void_p
+    p = L.make_params(1, 2, 128, 4, None, False, 0.0, L.LF_BF16)
+    rc = lib.lf_attn_decode(ctypes.byref(p), *([vp(a16)] * 5), None, None)
+    assert rc == L.LF_ERR_INVALID and b"causal" in lib.lf_attn_last_error()
+    pc = L.make_params(1, 2, 128, 4, None, True, 0.0, L.LF_BF16)
+    rc = lib.lf_attn_decode(ctypes.byref(pc), None, *([vp(a16)] * 4), None, None)
+    assert rc == L.LF_ERR_INVALID and b"q" in lib.lf_attn_last_error()
+    rc = lib.lf_attn_decode(ctypes.byref(pc), vp(a16), vp(a16 + 4), *([vp(a16)] * 3), None, None)
+    assert rc == L.LF_ERR_INVALID and b"aligned" in lib.lf_attn_last_error()

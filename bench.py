@@ -52,14 +52,22 @@ def _peaks():
 
 
 def algorithmic_bytes(wl, mask) -> int:
-    """Bytes one forward must move at least: Q_s, K_s, V_s read and O
-    written for every row, Q_g read at the global rows, K_g and V_g read in
-    full, the mask read and the fp32 log-normaliser written."""
+    """Bytes one forward must move at least, per sequence b and head:
+    Q_s, K_s, V_s read at the valid rows (mask != 0; a padding row is never
+    a query nor a key), Q_g read at the global rows, K_g and V_g read at the
+    valid rows only when the sequence has a global token (nothing else reads
+    them), O (every row, zeros at padding) and the fp32 log-normaliser
+    written, and the int32 mask read once."""
     eb = 4 if wl.dtype == "f32" else 2
     row = wl.head_dim * eb
-    nrows = wl.B * wl.H * wl.n
-    ng = int((mask == 2).sum())
-    return (4 * nrows * row + wl.H * ng * row + 2 * nrows * row + mask.size * 4 + nrows * 4)
+    total = mask.size * 4
+    for b in range(mask.shape[0]):
+        nvalid = int((mask[b] != 0).sum())
+        ng = int((mask[b] == 2).sum())
+        per_head = 3 * nvalid * row + ng * row + (2 * nvalid * row if ng else 0)
+        per_head += wl.n * row + wl.n * 4
+        total += wl.H * per_head
+    return total
 
 
 class ClockSampler:
@@ -157,6 +165,42 @@ def _dist():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return ws, rank, local
+
+
+def resolve_world(gpus: int, env=None):
+    """The rank layout for ``--gpus N``.  Under a launcher (torchrun sets
+    WORLD_SIZE) N must equal the world size.  Without one, N = 1 runs here
+    and N > 1 returns None: the caller relaunches itself with one process
+    per GPU (``launch_command``).  Returns (world, rank, local_rank)."""
+    env = os.environ if env is None else env
+    if gpus < 1:
+        raise SystemExit("bench.py: --gpus must be >= 1 (got %d)" % gpus)
+    if "WORLD_SIZE" in env:
+        world = int(env["WORLD_SIZE"])
+        if world != gpus:
+            raise SystemExit("bench.py: --gpus %d but the launcher started %d ranks" % (gpus, world))
+        return world, int(env.get("RANK", "0")), int(env.get("LOCAL_RANK", "0"))
+    if gpus == 1:
+        return 1, 0, 0
+    return None
+
+
+def launch_command(gpus: int, argv):
+    """torchrun command that reruns this script with one rank per GPU (local
+    rendezvous on 127.0.0.1)."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            "--nproc-per-node", str(gpus), "--master-addr", "127.0.0.1", "--master-port",
+            str(29500 + os.getpid() % 1000), os.path.abspath(__file__)] + list(argv)
+
+
+def rank_step_time(local_ms: float, world: int, device=None) -> float:
+    """Cross-rank part of a timed region: every rank has timed its own K
+    steps on its device; after a barrier the slowest rank's time is the
+    job's step time (the same on every rank)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    return max_over_ranks(local_ms, world, device)
 
 
 def run_reference(args, wl):
@@ -344,6 +388,10 @@ def main():
                     help="also time the backward (default for workloads with a backward)")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
+    layout = resolve_world(args.gpus)
+    if layout is None:
+        # --gpus N > 1 without a launcher: one process per GPU under torchrun
+        return subprocess.call(launch_command(args.gpus, sys.argv[1:]))
     if args.impl == "reference":
         return run_reference(args, wl)
 
@@ -352,7 +400,7 @@ def main():
 
     if args.decode:
         return run_decode(args, wl)
-    world, rank, local = _dist()
+    world, rank, local = layout
     if world > 1:
         import datetime
         import torch.distributed as dist
@@ -432,13 +480,12 @@ def main():
     L.lf_attn_set_timing_events(None, None)
     torch.cuda.synchronize(dev)
     launches = L.lf_attn_launch_count() - launches0
-    if world > 1:
-        torch.distributed.barrier()
     clocks = sampler.stop()
     t_ms = e0.elapsed_time(e1)
     k_ms = float(np.mean([a.elapsed_time(b) for a, b in kev]))
     att.status()
-    t_ms = max_over_ranks(t_ms, world, dev)
+    t_ms = rank_step_time(t_ms, world, dev)
+    k_ms = rank_step_time(k_ms, world, dev)
     ms_step_eager = t_ms / args.steps
     ms_step = ms_step_eager
     if not args.no_graph:
@@ -467,7 +514,7 @@ def main():
             graphs[k % nsets].replay()
         g1.record(stream)
         torch.cuda.synchronize(dev)
-        gt_ms = max_over_ranks(g0.elapsed_time(g1), world, dev)
+        gt_ms = rank_step_time(g0.elapsed_time(g1), world, dev)
         ms_step = gt_ms / args.steps
         att.status()
         del graphs
@@ -495,7 +542,7 @@ def main():
         o_host.copy_(d["o"], non_blocking=True)
     ee1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(ee0.elapsed_time(ee1) / e2e_steps, world, dev)
+    e2e_ms = rank_step_time(ee0.elapsed_time(ee1) / e2e_steps, world, dev)
     h2d = set_bytes + host["mask"].numel() * 4
     d2h = o_host.numel() * o_host.element_size()
 

@@ -173,11 +173,20 @@ int lf_attn_set_timing_events(void *ev_start, void *ev_stop);
  * call before any stream capture.  All calls on a device share the one
  * array, so calls that may overlap on the GPU (other streams, other host
  * threads) race and must be serialised by the caller.  The device status
- * word of this variant is not readable through lf_attn_status. */
+ * word of this variant lives in that array: read it with
+ * lf_attn_status_noalloc.  The cached address does not survive a
+ * cudaDeviceReset of the device; do not use this call after one. */
 int lf_attn_fwd_noalloc(const lf_attn_params *p, const void *q_s,
                         const void *k_s, const void *v_s, const void *q_g,
                         const void *k_g, const void *v_g, const int32_t *mask,
                         void *o, float *lse, void *stream);
+
+/* Synchronise `stream`, read and clear the device status word of the
+ * static scratch of lf_attn_fwd_noalloc on the current device.  Every
+ * lf_attn_fwd_noalloc clears that word when it starts, so this returns
+ * LF_OK or the first device-side error of the latest call on the device
+ * (codes as for lf_attn_status).  Allocates nothing. */
+int lf_attn_status_noalloc(void *stream);
 
 /* Number of kernels this library has launched in this process so far (all
  * threads).  Lets a caller count the kernels inside a timed region. */

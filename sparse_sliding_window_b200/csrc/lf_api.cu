@@ -9,6 +9,9 @@
 
 #include <algorithm>
 #include <atomic>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "lf_attn.h"
 #include "lf_common.cuh"
@@ -30,6 +33,40 @@ static int lf_fail(int code, const char *fmt, ...) {
 }
 
 int lf_record_error(int code, const char *msg) { return lf_fail(code, "%s", msg); }
+
+// Per-device launch state.  cudaFuncSetAttribute acts on the current
+// device's context only, and the SM count differs between devices, so both
+// are kept per (device ordinal, kernel), under one lock for callers on
+// several host threads.
+static std::mutex g_dev_mu;
+static std::map<std::pair<int, const void *>, int> g_smem_set;  // kernel -> bytes set
+static std::map<int, int> g_nsm;
+
+cudaError_t lf_kernel_smem(const void *fn, int smem_bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  auto key = std::make_pair(dev, fn);
+  auto it = g_smem_set.find(key);
+  if (it != g_smem_set.end() && it->second >= smem_bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e == cudaSuccess) g_smem_set[key] = smem_bytes;
+  return e;
+}
+
+int lf_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  auto it = g_nsm.find(dev);
+  if (it != g_nsm.end()) return it->second;
+  int nsm = 0;
+  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
+    nsm = 148;
+  g_nsm[dev] = nsm;
+  return nsm;
+}
 
 static int lf_cuda(cudaError_t e, const char *what) {
   if (e == cudaSuccess) return LF_OK;

@@ -151,6 +151,12 @@ __device__ __forceinline__ float2 lf_warp_sum2(float a, float b) {
 #define LF_LOG2E 1.4426950408889634f
 #define LF_LN2 0.6931471805599453f
 
+// Raise fn's dynamic shared-memory limit to smem_bytes on the current
+// device (once per device and kernel; thread-safe).
+cudaError_t lf_kernel_smem(const void *fn, int smem_bytes);
+// SM count of the current device (cached per device; thread-safe).
+int lf_sm_count();
+
 // process-wide count of kernel launches made by the library
 void lf_launches_add(int k);
 uint64_t lf_launches_get();

@@ -29,6 +29,37 @@ static void *g_static_addr[LF_STATIC_MAX_DEVICES];
 // defined in lf_api.cu: record an error for lf_attn_last_error()
 int lf_record_error(int code, const char *msg);
 
+// Device address of the static scratch on the current device; looked up
+// once per device (with that device current) and cached.
+static int lf_static_base(void **base, const char *who) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    char msg[128];
+    snprintf(msg, sizeof(msg), "%s: cudaGetDevice failed", who);
+    return lf_record_error(LF_ERR_CUDA, msg);
+  }
+  if (dev < 0 || dev >= LF_STATIC_MAX_DEVICES) {
+    char msg[128];
+    snprintf(msg, sizeof(msg), "%s: device ordinal out of range", who);
+    return lf_record_error(LF_ERR_UNSUPPORTED, msg);
+  }
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
+    // first use on this device (the current one): look the symbol up
+    void *ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, lf_static_ws);
+    if (e != cudaSuccess || !ptr) {
+      char msg[128];
+      snprintf(msg, sizeof(msg), "%s: cudaGetSymbolAddress failed", who);
+      return lf_record_error(LF_ERR_CUDA, msg);
+    }
+    g_static_addr[dev] = ptr;
+  }
+  *base = g_static_addr[dev];
+  return LF_OK;
+}
+
 extern "C" int lf_attn_fwd_noalloc(const lf_attn_params *p, const void *q_s, const void *k_s,
                                    const void *v_s, const void *q_g, const void *k_g,
                                    const void *v_g, const int32_t *mask, void *o, float *lse,
@@ -44,27 +75,21 @@ extern "C" int lf_attn_fwd_noalloc(const lf_attn_params *p, const void *q_s, con
              need, (size_t)LF_STATIC_WORKSPACE_BYTES);
     return lf_record_error(LF_ERR_UNSUPPORTED, msg);
   }
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return lf_record_error(LF_ERR_CUDA, "lf_attn_fwd_noalloc: cudaGetDevice failed");
-  if (dev < 0 || dev >= LF_STATIC_MAX_DEVICES)
-    return lf_record_error(LF_ERR_UNSUPPORTED, "lf_attn_fwd_noalloc: device ordinal out of range");
   void *base = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_static_mu);
-    if (!g_static_addr[dev]) {
-      // first call on this device (the current one): look the symbol up
-      void *ptr = nullptr;
-      e = cudaGetSymbolAddress(&ptr, lf_static_ws);
-      if (e != cudaSuccess || !ptr)
-        return lf_record_error(LF_ERR_CUDA, "lf_attn_fwd_noalloc: cudaGetSymbolAddress failed");
-      g_static_addr[dev] = ptr;
-    }
-    base = g_static_addr[dev];
-  }
+  const int st = lf_static_base(&base, "lf_attn_fwd_noalloc");
+  if (st != LF_OK) return st;
   // The regular forward clears the status word at its start and fully
   // writes every other scratch region before reading it, so the contents a
   // previous call left behind never matter.
   return lf_attn_fwd(p, q_s, k_s, v_s, q_g, k_g, v_g, mask, o, lse, base,
                      (size_t)LF_STATIC_WORKSPACE_BYTES, stream);
+}
+
+// The device status word of the static scratch: the same read-and-clear as
+// lf_attn_status, on the array of the current device.  Allocates nothing.
+extern "C" int lf_attn_status_noalloc(void *stream) {
+  void *base = nullptr;
+  const int st = lf_static_base(&base, "lf_attn_status_noalloc");
+  if (st != LF_OK) return st;
+  return lf_attn_status(base, stream);
 }

@@ -711,19 +711,15 @@ int lf_tc_bwd(const LfLaunch &L, const LfTcBwdArgs &a, char *err, size_t errlen)
       return LF_ERR_CUDA;
     }
   }
-  static bool attr_done[2][2] = {{false, false}, {false, false}};
   const unsigned grid = (unsigned)((long long)D.B * P.per_batch);
   for (int mode = 0; mode < 2; mode++) {  // 0: dK/dV (rows = keys), 1: dQ (rows = queries)
     void (*kern)(const LfBwParams) =
         f16 ? (mode ? lf_tc_bwd_kernel<1, 1> : lf_tc_bwd_kernel<1, 0>)
             : (mode ? lf_tc_bwd_kernel<0, 1> : lf_tc_bwd_kernel<0, 0>);
-    if (!attr_done[f16][mode]) {
-      ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LF_BW_SMEM);
-      if (ce != cudaSuccess) {
-        snprintf(err, errlen, "cudaFuncSetAttribute (backward): %s", cudaGetErrorString(ce));
-        return LF_ERR_CUDA;
-      }
-      attr_done[f16][mode] = true;
+    ce = lf_kernel_smem((const void *)kern, LF_BW_SMEM);
+    if (ce != cudaSuccess) {
+      snprintf(err, errlen, "cudaFuncSetAttribute (backward): %s", cudaGetErrorString(ce));
+      return LF_ERR_CUDA;
     }
     P.out0 = mode ? a.dqs : a.dvs;
     P.out1 = mode ? nullptr : a.dks;

@@ -24,7 +24,7 @@ ERROR_NAMES = {1: "LF_ERR_INVALID", 2: "LF_ERR_UNSUPPORTED", 3: "LF_ERR_CUDA",
 EXPORTS = ["lf_attn_version", "lf_attn_workspace_size", "lf_attn_fwd", "lf_attn_bwd",
            "lf_attn_count_pairs", "lf_attn_mask_dump", "lf_attn_status",
            "lf_attn_set_timing_events", "lf_attn_launch_count", "lf_attn_last_error",
-           "lf_attn_fwd_noalloc", "lf_attn_decode"]
+           "lf_attn_fwd_noalloc", "lf_attn_status_noalloc", "lf_attn_decode"]
 LF_STATIC_WORKSPACE_BYTES = 16 << 20
 
 
@@ -68,6 +68,8 @@ def load(path: str = LIB_PATH):
         lib.lf_attn_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         lib.lf_attn_decode.restype = i32
         lib.lf_attn_fwd_noalloc.restype = i32
+        lib.lf_attn_status_noalloc.argtypes = [vp]
+        lib.lf_attn_status_noalloc.restype = i32
         for f in ("fwd", "bwd", "count_pairs", "mask_dump", "status", "set_timing_events"):
             getattr(lib, "lf_attn_" + f).restype = i32
         _lib = lib
@@ -136,6 +138,12 @@ def lf_attn_fwd_noalloc(p, q_s, k_s, v_s, q_g, k_g, v_g, mask, o, lse, stream=No
     _check(load().lf_attn_fwd_noalloc(ctypes.byref(p), _ptr(q_s), _ptr(k_s), _ptr(v_s), _ptr(q_g),
                                       _ptr(k_g), _ptr(v_g), _ptr(mask), _ptr(o), _ptr(lse),
                                       _stream(stream)))
+
+
+def lf_attn_status_noalloc(stream=None):
+    """Read and clear the device status word of lf_attn_fwd_noalloc's static
+    scratch on the current device (raises LfError on a device-side error)."""
+    _check(load().lf_attn_status_noalloc(_stream(stream)))
 
 
 def lf_attn_decode(p, q, k_cache, v_cache, lengths, o, lse=None, stream=None):

@@ -75,3 +75,34 @@ def test_algorithmic_bytes_of_base_workload():
     expect = 4 * rows * 128 + 12 * 65 * 128 + 2 * rows * 128 + 4096 * 4 + rows * 4
     assert expect == 38061568
     assert bench.algorithmic_bytes(wl, mask) == expect
+
+
+def test_algorithmic_bytes_of_charlm_workload():
+    """Counted by hand: no global token, so K_g / V_g / Q_g are never read;
+    8 heads x 23040 valid rows of 128 bytes for Q_s, K_s, V_s read and O
+    written, the fp32 log-normaliser of every row and the int32 mask."""
+    sys.path.insert(0, ROOT)
+    import bench
+    wl = synth.WORKLOADS["charlm_bf16"]
+    mask = synth.make_inputs(wl, with_do=False)["mask"]
+    rows = 8 * 23040
+    expect = 4 * rows * 128 + rows * 4 + 23040 * 4
+    assert expect == 95201280
+    assert bench.algorithmic_bytes(wl, mask) == expect
+
+
+def test_algorithmic_bytes_of_batched_workload():
+    """Counted by hand from the seeded structure: the 8 sequences hold
+    25229 valid tokens in all, each with 17 global tokens; per head, Q_s /
+    K_s / V_s / K_g / V_g are read at the valid rows (every sequence has a
+    global token), Q_g at the 136 global rows, O and the log-normaliser are
+    written for all 8 x 4096 rows, and the mask is read once."""
+    sys.path.insert(0, ROOT)
+    import bench
+    wl = synth.WORKLOADS["batched_f16"]
+    mask = synth.make_inputs(wl, with_do=False)["mask"]
+    assert int((mask != 0).sum()) == 25229 and int((mask == 2).sum()) == 136
+    expect = (5 * 12 * 25229 * 128 + 12 * 136 * 128 + 12 * 8 * 4096 * 128 + 12 * 8 * 4096 * 4
+              + 8 * 4096 * 4)
+    assert expect == 246003200
+    assert bench.algorithmic_bytes(wl, mask) == expect

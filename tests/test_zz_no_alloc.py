@@ -6,6 +6,12 @@ shared array -- with different masks, shapes and inputs -- match the regular
 workspace entry point within the tolerances of the other parity tests, and
 that a problem too large for the array is refused up front.
 
+The array also holds the call's device status word, read through
+lf_attn_status_noalloc: a mask value outside {0, 1, 2} must come back as
+LF_ERR_DEVICE_INPUT there, and the next good call must come back clean (each
+call clears the word).  Free device memory is compared around the calls: the
+entry point exists so that nothing is allocated, so it must not drop.
+
 Collected last on purpose (file name), so a run that stops at the first
 failure has already run every other test.
 """
@@ -46,14 +52,53 @@ def test_noalloc_matches_workspace_forward_two_calls():
     m2[1, 500:] = 0
     m2[1, [3, 90]] = 2
     cases = [(1, 3, 1000, 64, [1, 2, 1], m1, 21, "bf16"), (2, 2, 700, 100, [1, 1], m2, 22, "f16")]
-    for B, H, n, r, dil, m, seed, dt in cases:   # two calls in a row on the shared scratch
-        p, g, o_ref, lse_ref = _case(B, H, n, r, dil, m, seed, dt)
-        o = torch.full_like(o_ref, float("nan"))
-        lse = torch.full_like(lse_ref, float("nan"))
+    prepared = [_case(*c) for c in cases]
+    outs = [(torch.full_like(o_ref, float("nan")), torch.full_like(lse_ref, float("nan")))
+            for _, _, o_ref, lse_ref in prepared]
+    # warm-up calls: the library's device code (and with it the static array)
+    # may be loaded lazily, kernel by kernel, on first use
+    for (p, g, _, _), (o, lse) in zip(prepared, outs):
         L.lf_attn_fwd_noalloc(p, g["qs"], g["ks"], g["vs"], g["qg"], g["kg"], g["vg"], g["mask"], o, lse)
+        L.lf_attn_status_noalloc()
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for (p, g, _, _), (o, lse) in zip(prepared, outs):   # two calls in a row on the shared scratch
+        o.fill_(float("nan"))
+        lse.fill_(float("nan"))
         torch.cuda.synchronize()
+        free_before = torch.cuda.mem_get_info()[0]
+        L.lf_attn_fwd_noalloc(p, g["qs"], g["ks"], g["vs"], g["qg"], g["kg"], g["vg"], g["mask"], o, lse)
+        L.lf_attn_status_noalloc()
+        torch.cuda.synchronize()
+        assert torch.cuda.mem_get_info()[0] == free_before  # nothing allocated by the call
+    assert torch.cuda.mem_get_info()[0] == free0
+    for (p, g, o_ref, lse_ref), (o, lse), c in zip(prepared, outs, cases):
+        dt = c[-1]
         U.compare("noalloc/o", U.to_f64(o), U.to_f64(o_ref), dt)
         U.compare_lse(U.to_f64(lse), U.to_f64(lse_ref), dt)
+
+
+def test_noalloc_status_reports_device_input_errors_then_clears():
+    import torch
+    lfbuild.build()
+    L.load()
+    m = np.ones((1, 500), np.int32)
+    m[0, 0] = 2
+    p, g, o_ref, lse_ref = _case(1, 2, 500, 32, [1, 1], m, 31)
+    bad = g["mask"].clone()
+    bad[0, 123] = 3                      # not a mask code: only the device sees it
+    o = torch.empty_like(o_ref)
+    lse = torch.empty_like(lse_ref)
+    L.lf_attn_fwd_noalloc(p, g["qs"], g["ks"], g["vs"], g["qg"], g["kg"], g["vg"], bad, o, lse)
+    with pytest.raises(L.LfError) as e:
+        L.lf_attn_status_noalloc()
+    assert e.value.code == L.LF_ERR_DEVICE_INPUT
+    # the next good call starts from a clear status word and matches
+    L.lf_attn_fwd_noalloc(p, g["qs"], g["ks"], g["vs"], g["qg"], g["kg"], g["vg"], g["mask"], o, lse)
+    L.lf_attn_status_noalloc()
+    torch.cuda.synchronize()
+    U.compare("noalloc/o after error", U.to_f64(o), U.to_f64(o_ref), "bf16")
+    U.compare_lse(U.to_f64(lse), U.to_f64(lse_ref), "bf16")
 
 
 def test_noalloc_refuses_problems_larger_than_its_scratch():

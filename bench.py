@@ -266,12 +266,14 @@ def cpu_baseline(wl, budget_s=10.0):
             "sample": "%d of %d (b,h) heads of %s, float64, %.1f s" % (done, wl.B * wl.H, wl.name, t_total)}
 
 
-def time_backward(att, d, wl, pairs, world, args, dev, stream):
+def time_backward(att, d, wl, pairs, world, steps, warmup, dev, stream):
     """Time lf_attn_bwd (six gradients) on the forward's outputs; reported
     beside the forward metric (algorithmic 8 * head_dim FLOP per pair)."""
     import torch
     from sparse_sliding_window_b200 import lf_attn as L
-    g = torch.randn_like(d["qs"])
+    g = d.get("do")
+    if g is None:
+        g = torch.randn_like(d["qs"])
     if att.ws_b is None:
         att.ws_b = L.workspace(att.p, True, dev)
     grads = [torch.empty_like(d["qs"]) for _ in range(6)]
@@ -280,11 +282,11 @@ def time_backward(att, d, wl, pairs, world, args, dev, stream):
         L.lf_attn_bwd(att.p, d["qs"], d["ks"], d["vs"], d["qg"], d["kg"], d["vg"], d["mask"], d["o"],
                       d["lse"], g, *grads, att.ws_b)
 
-    for _ in range(max(3, args.warmup // 4)):
+    for _ in range(max(3, warmup // 4)):
         bstep()
     torch.cuda.synchronize(dev)
     att.status(bwd=True)
-    k = max(3, min(args.steps, 20))
+    k = max(3, min(steps, 20))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
@@ -293,28 +295,29 @@ def time_backward(att, d, wl, pairs, world, args, dev, stream):
         bstep()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = max_over_ranks(e0.elapsed_time(e1) / k, world, dev)
+    att.status(bwd=True)
+    ms = rank_step_time(e0.elapsed_time(e1) / k, world, dev)
     kinds = ("CUDA-core backward (delta, dQ, dK_s/dV_s, dK_g/dV_g)" if wl.dtype == "f32" else
              "tensor-core dQ and dK/dV band kernels + CUDA-core global-token parts")
-    return {"ms_per_step": ms, "steps": k, "kernels": kinds,
-            "tflops_algorithmic": 8.0 * wl.head_dim * pairs * world / (ms * 1e-3) / 1e12,
+    pk = _peaks()
+    tfl = 8.0 * wl.head_dim * pairs * world / (ms * 1e-3) / 1e12
+    return {"ms_per_step": ms, "steps": k, "kernels": kinds, "launch": "eager",
+            "tflops_algorithmic": tfl, "tensor_frac_sustained": tfl / pk["bf16_sus"],
             "scores_per_s": pairs * world / (ms * 1e-3)}
 
 
-def run_decode(args, wl):
+def decode_numbers(wl, steps, warmup, dev):
     """Decode step of a causal workload: one new token per sequence against
-    the full-length cache (every head), timed on the device.  HBM-bound:
-    the window's key and value rows are read once per head."""
+    the full-length cache (every head), timed on the device over CUDA-graph
+    replays.  HBM-bound: the window's key and value rows are read once per
+    head.  Returns the numbers and the roofline."""
     import torch
     from sparse_sliding_window_b200 import lf_attn as L
     assert wl.causal, "the decode step is the causal window"
-    dev = torch.device("cuda", 0)
     inp = synth.make_inputs(wl, with_do=False)
-    tdt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[wl.dtype]
 
     def dev_t(a):
-        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if wl.dtype == "bf16" else torch.from_numpy(a)
-        return t.to(dev)
+        return _host_tensor(a, wl.dtype).to(dev)
     kc, vc = dev_t(inp["ks"]), dev_t(inp["vs"])
     q = dev_t(np.ascontiguousarray(inp["qs"][:, :, -1]))
     lens = torch.full((wl.B,), wl.n, dtype=torch.int32, device=dev)
@@ -322,7 +325,7 @@ def run_decode(args, wl):
     lse = torch.empty((wl.B, wl.H), dtype=torch.float32, device=dev)
     p = L.make_params(wl.B, wl.H, wl.n, wl.r, wl.dilation, True, 0.0,
                       {"bf16": L.LF_BF16, "f16": L.LF_F16, "f32": L.LF_F32}[wl.dtype])
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         L.lf_attn_decode(p, q, kc, vc, lens, o, lse)
     torch.cuda.synchronize(dev)
     # a serving loop replays the step from a CUDA graph: the host launches
@@ -339,7 +342,7 @@ def run_decode(args, wl):
     with torch.cuda.graph(gr):
         for _ in range(per_graph):
             L.lf_attn_decode(p, q, kc, vc, lens, o, lse)
-    reps = max(1, args.steps // per_graph)
+    reps = max(1, steps // per_graph)
     for _ in range(3):
         gr.replay()
     torch.cuda.synchronize(dev)
@@ -355,19 +358,209 @@ def run_decode(args, wl):
     keys = sum(min(wl.r, (wl.n - 1) // d) + 1 for d in wl.dilation) * wl.B
     nbytes = keys * 2 * 64 * eb + 2 * wl.B * wl.H * 64 * eb + wl.B * wl.H * 4
     pk = _peaks()
-    line = {"metric": "decode tokens/s (causal window, one new token per sequence, all heads)",
-            "value": wl.B / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": wl.dtype,
-            "steps_timed": reps * per_graph,
-            "data": "synthetic", "config": {"workload": wl.name + " decode", "B": wl.B, "H": wl.H,
-                                            "cache_len": wl.n, "window_one_sided": wl.r,
-                                            "dilation": wl.dilation},
+    return {"ms_per_step": ms, "tokens_per_s": wl.B / (ms * 1e-3), "steps_timed": reps * per_graph,
+            "launch": "cuda_graph",
             "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": pk["hbm"],
                          "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm"],
                          "traffic": None, "algorithmic_bytes": nbytes,
                          "note": "CUDA-graph replay of 32 steps; a step still includes the device-side launch gap"}}
+
+
+def run_decode(args, wl):
+    import torch
+    dev = torch.device("cuda", 0)
+    d = decode_numbers(wl, args.steps, args.warmup, dev)
+    line = {"metric": "decode tokens/s (causal window, one new token per sequence, all heads)",
+            "value": d["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": d["ms_per_step"], "higher_is_better": True,
+            "dtype": wl.dtype, "steps_timed": d["steps_timed"], "data": "synthetic",
+            "config": {"workload": wl.name + " decode", "B": wl.B, "H": wl.H, "cache_len": wl.n,
+                       "window_one_sided": wl.r, "dilation": wl.dilation},
+            "roofline": d["roofline"]}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def _host_tensor(a, dtype):
+    import torch
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a))
+
+
+NAMES = ["qs", "ks", "vs", "qg", "kg", "vg"]
+
+
+def measure(wl, kern, steps, warmup, world, dev, stream, graph=True, e2e=False,
+            min_warm_seconds=0.0, sampler=None):
+    """One workload's forward on this rank: attended pairs (the library's
+    pair counter), the CUDA-graph and eager step times over input sets that
+    rotate through more than the L2 cache, the main kernel's time from CUDA
+    events the library records around it on its stream, the roofline of
+    that kernel, and optionally the end-to-end time through the public API
+    with host buffers.  Timed regions end with a barrier and the max over
+    ranks."""
+    import torch
+    from sparse_sliding_window_b200 import lf_attn as L
+    inp = synth.make_inputs(wl, with_do=wl.backward)
+    mask_np = inp["mask"]
+    ng = int((mask_np == 2).sum(axis=1).max())
+    att = L.LongformerAttention(wl.B, wl.H, wl.n, wl.r, wl.dilation, wl.causal, dtype=wl.dtype,
+                                max_global=ng, kernel=kern, device=dev)
+    host = {k: _host_tensor(inp[k], wl.dtype).pin_memory() for k in NAMES}
+    host["mask"] = torch.from_numpy(mask_np).pin_memory()
+    set_bytes = sum(host[k].numel() * host[k].element_size() for k in NAMES)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    nsets = max(2, int(math.ceil(1.5 * l2 / max(set_bytes, 1))) + 1)
+    sets = []
+    for s in range(nsets):
+        d = {k: host[k].to(dev, non_blocking=False) for k in NAMES + ["mask"]}
+        d["o"] = torch.empty_like(d["qs"])
+        d["lse"] = torch.empty(d["qs"].shape[:3], dtype=torch.float32, device=dev)
+        sets.append(d)
+    if wl.backward:
+        sets[0]["do"] = _host_tensor(inp["do"], wl.dtype).to(dev)
+    torch.cuda.synchronize(dev)
+    pairs = int(att.count_pairs(sets[0]["mask"]).sum().item())
+    att.status()
+
+    def step(i):
+        d = sets[i % nsets]
+        att.fwd(d["qs"], d["ks"], d["vs"], d["qg"], d["kg"], d["vg"], d["mask"], d["o"], d["lse"])
+
+    if sampler is not None:
+        sampler.start()
+    i = 0
+    t_start = time.time()
+    while i < warmup or time.time() - t_start < min_warm_seconds:
+        step(i)
+        i += 1
+        if i % 64 == 0:
+            torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(dev)
+    att.status()
+    # eager steps, with the kernel events of every step
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b in kev:  # create the CUDA events; the library re-records them
+        a.record(stream)
+        b.record(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = L.lf_attn_launch_count()
+    e0.record(stream)
+    for k in range(steps):
+        L.lf_attn_set_timing_events(*kev[k])
+        step(i + k)
+    e1.record(stream)
+    L.lf_attn_set_timing_events(None, None)
+    torch.cuda.synchronize(dev)
+    launches = L.lf_attn_launch_count() - launches0
+    clocks = sampler.stop() if sampler is not None else None
+    att.status()
+    t_ms = rank_step_time(e0.elapsed_time(e1), world, dev)
+    k_ms = rank_step_time(float(np.mean([a.elapsed_time(b) for a, b in kev])), world, dev)
+    ms_step_eager = t_ms / steps
+    ms_step = ms_step_eager
+    if graph:
+        # the same steps replayed from CUDA graphs (one per input set): the
+        # library's launches are captured once, replays skip host launch cost
+        graphs = []
+        for sidx in range(nsets):
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                step(sidx)
+            stream.wait_stream(side)
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                step(sidx)
+            graphs.append(gr)
+        for k in range(max(3, warmup)):
+            graphs[k % nsets].replay()
+        torch.cuda.synchronize(dev)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        g0.record(stream)
+        for k in range(steps):
+            graphs[k % nsets].replay()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_step = rank_step_time(g0.elapsed_time(g1), world, dev) / steps
+        att.status()
+        del graphs
+    flops = 4.0 * wl.head_dim * pairs
+    pk = _peaks()
+    abytes = algorithmic_bytes(wl, mask_np)
+    t_flop = flops / (pk["bf16"] * 1e12)
+    t_byte = abytes / (pk["hbm"] * 1e9)
+    k_s = k_ms * 1e-3
+    if t_byte >= t_flop:
+        roof = {"bound": "hbm", "achieved": abytes / k_s / 1e9, "peak": pk["hbm"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / k_s / 1e12, "peak": pk["bf16"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = kernel_traffic(wl.name) if kern != 1 else None
+    roof["peak_source"] = pk["src"]
+    roof["kernel_ms"] = k_ms
+    roof["algorithmic_bytes"] = abytes
+    roof["algorithmic_flops"] = flops
+    roof["tensor_view"] = {"achieved_tflops": flops / k_s / 1e12, "peak": pk["bf16"],
+                           "frac": flops / k_s / 1e12 / pk["bf16"]}
+    roof["step_frac"] = max(t_flop, t_byte) / (ms_step * 1e-3)
+    roof["timed_on"] = "eager launches, events around the kernel on its stream"
+    out = {"wl": wl, "pairs": pairs, "ng": ng, "nsets": nsets, "set_bytes": set_bytes, "l2": l2,
+           "ms_step": ms_step, "ms_step_eager": ms_step_eager, "kernel_ms": k_ms,
+           "launches_per_step": launches / steps, "launches": launches, "roofline": roof,
+           "clocks": clocks, "scores_per_s": job_throughput(pairs, world, ms_step),
+           "tflops": flops * world / (ms_step * 1e-3) / 1e12, "att": att, "sets": sets}
+    if e2e:
+        # end-to-end through the public API: H2D of the step's inputs from
+        # pinned host memory, the forward, D2H of the output
+        o_host = torch.empty(sets[0]["o"].shape, dtype=sets[0]["o"].dtype).pin_memory()
+        d = sets[0]
+        for _ in range(3):
+            for k in NAMES + ["mask"]:
+                d[k].copy_(host[k], non_blocking=True)
+            att.fwd(d["qs"], d["ks"], d["vs"], d["qg"], d["kg"], d["vg"], d["mask"], d["o"], d["lse"])
+            o_host.copy_(d["o"], non_blocking=True)
+        torch.cuda.synchronize(dev)
+        ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_steps = max(3, min(steps, 50))
+        ee0.record(stream)
+        for _ in range(e2e_steps):
+            for k in NAMES + ["mask"]:
+                d[k].copy_(host[k], non_blocking=True)
+            att.fwd(d["qs"], d["ks"], d["vs"], d["qg"], d["kg"], d["vg"], d["mask"], d["o"], d["lse"])
+            o_host.copy_(d["o"], non_blocking=True)
+        ee1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = rank_step_time(ee0.elapsed_time(ee1) / e2e_steps, world, dev)
+        out["e2e"] = {"value": job_throughput(pairs, world, e2e_ms), "unit": UNIT,
+                      "h2d_bytes_per_step": int(set_bytes + host["mask"].numel() * 4),
+                      "d2h_bytes_per_step": int(o_host.numel() * o_host.element_size()),
+                      "ms_per_step": e2e_ms}
+    return out
+
+
+def summary(m):
+    """The per-workload numbers reported beside the headline line."""
+    wl, r = m["wl"], m["roofline"]
+    return {"step_ms": m["ms_step"], "step_ms_eager": m["ms_step_eager"], "kernel_ms": m["kernel_ms"],
+            "scores_per_s": m["scores_per_s"], "tflops": m["tflops"],
+            "attended_pairs": m["pairs"], "dtype": wl.dtype,
+            "roofline": {"bound": r["bound"], "achieved": r["achieved"], "peak": r["peak"],
+                         "unit": r["unit"], "frac": r["frac"], "step_frac": r["step_frac"],
+                         "algorithmic_bytes": r["algorithmic_bytes"], "traffic": r["traffic"],
+                         "tensor_frac": r["tensor_view"]["frac"]},
+            "gpu_launches_per_step": m["launches_per_step"],
+            "config": {"B": wl.B, "H": wl.H, "n": wl.n, "window": 2 * wl.r,
+                       "dilation": sorted(set(wl.dilation)), "causal": wl.causal,
+                       "global_tokens_per_seq": m["ng"]}}
 
 
 def main():
@@ -386,6 +579,8 @@ def main():
                     help="time the causal-window decode step instead (causal workloads)")
     ap.add_argument("--bwd", action="store_true",
                     help="also time the backward (default for workloads with a backward)")
+    ap.add_argument("--no-others", action="store_true",
+                    help="skip the other workloads reported under 'workloads'")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
     layout = resolve_world(args.gpus)
@@ -412,177 +607,51 @@ def main():
     stream = torch.cuda.current_stream(dev)
     kern = {"auto": L.LF_KERNEL_AUTO, "simt": L.LF_KERNEL_SIMT, "tc": L.LF_KERNEL_TC}[args.kernel]
 
-    inp = synth.make_inputs(wl, with_do=False)
-    mask_np = inp["mask"]
-    ng = int((mask_np == 2).sum(axis=1).max())
-    att = L.LongformerAttention(wl.B, wl.H, wl.n, wl.r, wl.dilation, wl.causal, dtype=wl.dtype,
-                                max_global=ng, kernel=kern, device=dev)
-    tdt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[wl.dtype]
-
-    def host_tensor(a):
-        if wl.dtype == "bf16":
-            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
-        return torch.from_numpy(a)
-
-    names = ["qs", "ks", "vs", "qg", "kg", "vg"]
-    host = {k: host_tensor(inp[k]).pin_memory() for k in names}
-    host["mask"] = torch.from_numpy(mask_np).pin_memory()
-    set_bytes = sum(host[k].numel() * host[k].element_size() for k in names)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    nsets = max(2, int(math.ceil(1.5 * l2 / max(set_bytes, 1))) + 1)
-    sets = []
-    for s in range(nsets):
-        d = {k: host[k].to(dev, non_blocking=False) for k in names + ["mask"]}
-        d["o"] = torch.empty_like(d["qs"])
-        d["lse"] = torch.empty(d["qs"].shape[:3], dtype=torch.float32, device=dev)
-        sets.append(d)
-    torch.cuda.synchronize(dev)
-
-    # attended pairs of one step, from the library's pair counter (exact
-    # against the oracle in tests/)
-    pairs = int(att.count_pairs(sets[0]["mask"]).sum().item())
-    att.status()
-
-    def step(i):
-        d = sets[i % nsets]
-        att.fwd(d["qs"], d["ks"], d["vs"], d["qg"], d["kg"], d["vg"], d["mask"], d["o"], d["lse"])
-
-    # warm-up (count-based, stretched to >= min_warm_seconds for the clock samples)
     sampler = ClockSampler(getattr(torch.cuda.get_device_properties(dev), "uuid", None) and
                            "GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
-    sampler.start()
-    i = 0
-    t_start = time.time()
-    while i < args.warmup or time.time() - t_start < args.min_warm_seconds:
-        step(i)
-        i += 1
-        if i % 64 == 0:
-            torch.cuda.synchronize(dev)
-    torch.cuda.synchronize(dev)
-    att.status()
-
-    # kernel timing events (main attention kernel of every timed step)
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for a, b in kev:  # create the CUDA events; the library re-records them
-        a.record(stream)
-        b.record(stream)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    launches0 = L.lf_attn_launch_count()
-    e0.record(stream)
-    for k in range(args.steps):
-        L.lf_attn_set_timing_events(*kev[k])
-        step(i + k)
-    e1.record(stream)
-    L.lf_attn_set_timing_events(None, None)
-    torch.cuda.synchronize(dev)
-    launches = L.lf_attn_launch_count() - launches0
-    clocks = sampler.stop()
-    t_ms = e0.elapsed_time(e1)
-    k_ms = float(np.mean([a.elapsed_time(b) for a, b in kev]))
-    att.status()
-    t_ms = rank_step_time(t_ms, world, dev)
-    k_ms = rank_step_time(k_ms, world, dev)
-    ms_step_eager = t_ms / args.steps
-    ms_step = ms_step_eager
-    if not args.no_graph:
-        # the same steps replayed from CUDA graphs (one per input set): the
-        # library's launches are captured once, replays skip host launch cost
-        graphs = []
-        for sidx in range(nsets):
-            side = torch.cuda.Stream(dev)
-            side.wait_stream(stream)
-            with torch.cuda.stream(side):
-                step(sidx)
-            stream.wait_stream(side)
-            gr = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gr):
-                step(sidx)
-            graphs.append(gr)
-        for k in range(max(3, args.warmup)):
-            graphs[k % nsets].replay()
-        torch.cuda.synchronize(dev)
-        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize(dev)
-        g0.record(stream)
-        for k in range(args.steps):
-            graphs[k % nsets].replay()
-        g1.record(stream)
-        torch.cuda.synchronize(dev)
-        gt_ms = rank_step_time(g0.elapsed_time(g1), world, dev)
-        ms_step = gt_ms / args.steps
-        att.status()
-        del graphs
-    value = job_throughput(pairs, world, ms_step)
-    flops = 4.0 * wl.head_dim * pairs
-    tflops = flops * world / (ms_step * 1e-3) / 1e12
-
-    # end-to-end through the public API: H2D of the step's inputs from pinned
-    # host memory, the forward, D2H of the output
-    o_host = torch.empty(sets[0]["o"].shape, dtype=tdt).pin_memory()
-    d = sets[0]
-    for _ in range(3):
-        for k in names + ["mask"]:
-            d[k].copy_(host[k], non_blocking=True)
-        att.fwd(d["qs"], d["ks"], d["vs"], d["qg"], d["kg"], d["vg"], d["mask"], d["o"], d["lse"])
-        o_host.copy_(d["o"], non_blocking=True)
-    torch.cuda.synchronize(dev)
-    ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(3, min(args.steps, 50))
-    ee0.record(stream)
-    for _ in range(e2e_steps):
-        for k in names + ["mask"]:
-            d[k].copy_(host[k], non_blocking=True)
-        att.fwd(d["qs"], d["ks"], d["vs"], d["qg"], d["kg"], d["vg"], d["mask"], d["o"], d["lse"])
-        o_host.copy_(d["o"], non_blocking=True)
-    ee1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = rank_step_time(ee0.elapsed_time(ee1) / e2e_steps, world, dev)
-    h2d = set_bytes + host["mask"].numel() * 4
-    d2h = o_host.numel() * o_host.element_size()
-
-    pk = _peaks()
-    abytes = algorithmic_bytes(wl, mask_np)
-    t_flop = flops / (pk["bf16"] * 1e12)
-    t_byte = abytes / (pk["hbm"] * 1e9)
-    k_s = k_ms * 1e-3
-    if t_byte >= t_flop:
-        roof = {"bound": "hbm", "achieved": abytes / k_s / 1e9, "peak": pk["hbm"], "unit": "GB/s"}
-    else:
-        roof = {"bound": "tensor", "achieved": flops / k_s / 1e12, "peak": pk["bf16"], "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = kernel_traffic(wl.name) if args.kernel != "simt" else None
-    roof["peak_source"] = pk["src"]
-    roof["kernel_ms"] = k_ms
-    roof["algorithmic_bytes"] = abytes
-    roof["algorithmic_flops"] = flops
-    roof["tensor_view"] = {"achieved_tflops": flops / k_s / 1e12, "peak": pk["bf16"],
-                           "frac": flops / k_s / 1e12 / pk["bf16"]}
-    roof["step_frac"] = max(t_flop, t_byte) / (ms_step * 1e-3)
-    roof["timed_on"] = "eager launches, events around the kernel on its stream"
-
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "ms_per_step_eager": ms_step_eager,
+    m = measure(wl, kern, args.steps, args.warmup, world, dev, stream, graph=not args.no_graph,
+                e2e=True, min_warm_seconds=args.min_warm_seconds, sampler=sampler)
+    pairs = m["pairs"]
+    line = {"metric": METRIC, "value": m["scores_per_s"], "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": m["ms_step"],
+            "ms_per_step_eager": m["ms_step_eager"],
             "launch": "eager" if args.no_graph else "cuda_graph", "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
             "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "n": wl.n, "window": 2 * wl.r,
                        "head_dim": wl.head_dim, "dilation": sorted(set(wl.dilation)),
-                       "causal": wl.causal, "global_tokens_per_seq": ng, "kernel": args.kernel,
+                       "causal": wl.causal, "global_tokens_per_seq": m["ng"], "kernel": args.kernel,
                        "l2": "inputs rotate over %d buffer sets (%.0f MB > L2 %.0f MB)" % (
-                           nsets, nsets * set_bytes / 1e6, l2 / 1e6),
+                           m["nsets"], m["nsets"] * m["set_bytes"] / 1e6, m["l2"] / 1e6),
                        "parallelism": "replicas x%d" % world if world > 1 else "1 GPU"},
-            "tflops": tflops, "attended_pairs_per_step": pairs * world,
-            "roofline": roof, "clocks": clocks, "gpu_launches": int(launches),
-            "e2e": {"value": pairs * world / (e2e_ms * 1e-3), "unit": UNIT,
-                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                    "ms_per_step": e2e_ms}}
+            "tflops": m["tflops"], "attended_pairs_per_step": pairs * world,
+            "roofline": m["roofline"], "clocks": m["clocks"], "gpu_launches": int(m["launches"]),
+            "e2e": m["e2e"]}
     if args.bwd or wl.backward:
-        line["backward"] = time_backward(att, sets[0], wl, pairs, world, args, dev, stream)
+        line["backward"] = time_backward(m["att"], m["sets"][0], wl, pairs, world, args.steps,
+                                         args.warmup, dev, stream)
+    del m
+    if not args.no_others and args.kernel != "simt":
+        # every other workload, driver-observed beside the headline: its
+        # forward step / main kernel / roofline, the backward where it has
+        # one, and the decode step of the causal one
+        others = {}
+        ksteps, kwarm = max(3, min(args.steps, 30)), max(3, min(args.warmup, 5))
+        for name in sorted(synth.WORKLOADS):
+            if name == wl.name:
+                continue
+            owl = synth.WORKLOADS[name]
+            om = measure(owl, kern, ksteps, kwarm, world, dev, stream, graph=not args.no_graph)
+            entry = summary(om)
+            entry["steps"] = ksteps
+            if owl.backward:
+                entry["backward"] = time_backward(om["att"], om["sets"][0], owl, om["pairs"], world,
+                                                  ksteps, kwarm, dev, stream)
+            if owl.causal:
+                entry["decode"] = decode_numbers(owl, 256, 3, dev)
+            others[name] = entry
+            del om
+            torch.cuda.empty_cache()
+        line["workloads"] = others
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:

@@ -157,6 +157,22 @@ int lf_attn_status(void *workspace, void *stream);
  * Pass NULL, NULL to turn it off. */
 int lf_attn_set_timing_events(void *ev_start, void *ev_stop);
 
+/* Test hook for the device-side failure detection (SURVEY: failure
+ * detection without a GPU fault).  Applies to the following lf_attn_fwd /
+ * lf_attn_bwd calls of the calling thread until it is called again:
+ *   wait_limit_us  the limit of every bounded device wait, in microseconds
+ *                  (0 = the default 1.5 s);
+ *   skip_kv_tile   > 0: CTA 0 of the tensor-core forward does not load the
+ *                  K/V tile of its tile stream number skip_kv_tile - 1, so the
+ *                  MMA warp's wait for it expires; the CTA records
+ *                  LF_ERR_DEVICE_TIMEOUT in the status word, lets its issued
+ *                  copies and MMAs finish, frees its TMEM and exits (outputs of
+ *                  that call are undefined).  0 = off.
+ * Nothing faults, traps or hangs; the context stays usable.  Pass 0, 0 to
+ * restore normal operation.  Returns LF_ERR_INVALID for a limit above 60 s
+ * or a negative tile. */
+int lf_attn_set_test_hooks(uint32_t wait_limit_us, int skip_kv_tile);
+
 /* Bytes of device scratch built into the library for lf_attn_fwd_noalloc. */
 #define LF_STATIC_WORKSPACE_BYTES (16u << 20)
 

@@ -23,6 +23,7 @@ static std::atomic<uint64_t> g_launches{0};
 void lf_launches_add(int k) { g_launches.fetch_add((uint64_t)k, std::memory_order_relaxed); }
 uint64_t lf_launches_get() { return g_launches.load(std::memory_order_relaxed); }
 static thread_local cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
+static thread_local int g_test_wait_us = 0, g_test_skip_tile = 0;
 
 static int lf_fail(int code, const char *fmt, ...) {
   va_list ap;
@@ -78,6 +79,15 @@ extern "C" int lf_attn_version(void) { return 1; }
 extern "C" uint64_t lf_attn_launch_count(void) { return lf_launches_get(); }
 
 extern "C" const char *lf_attn_last_error(void) { return g_err; }
+
+extern "C" int lf_attn_set_test_hooks(uint32_t wait_limit_us, int skip_kv_tile) {
+  g_err[0] = 0;
+  if (wait_limit_us > 60000000u) return lf_fail(LF_ERR_INVALID, "wait limit above 60 s");
+  if (skip_kv_tile < 0) return lf_fail(LF_ERR_INVALID, "skip_kv_tile must be >= 0");
+  g_test_wait_us = (int)wait_limit_us;
+  g_test_skip_tile = skip_kv_tile;
+  return LF_OK;
+}
 
 extern "C" int lf_attn_set_timing_events(void *ev_start, void *ev_stop) {
   g_ev_start = (cudaEvent_t)ev_start;
@@ -136,31 +146,37 @@ static int lf_prepare(const lf_attn_params *p, int for_bwd, LfDev &dev, LfWs &ws
 
   const size_t B = p->B, H = p->H, eb = lf_dtype_bytes(p->dtype);
   const size_t Ga = std::max(G, 1), Gka = std::max(dev.Gk, 16);
+  const bool tc = p->dtype != LF_F32 && p->kernel != LF_KERNEL_SIMT;
   size_t off = 0;
   ws.status = off;
-  off = lf_align(off + LF_ST_WORDS * 4);
+  {
+    size_t words = LF_ST_WORDS;
+    if (tc && !for_bwd) words += B * H * (((size_t)G + LF_BQ - 1) / LF_BQ);  // split counters
+    ws.status_bytes = words * 4;
+    off = lf_align(off + ws.status_bytes);
+  }
   ws.binfo = off;
   off = lf_align(off + B * LF_BI_WORDS * 4);
   ws.gidx = off;
   off = lf_align(off + B * Ga * 4);
   ws.grank = off;
   off = lf_align(off + B * ((size_t)n + 1) * 4);
-  const bool tc = p->dtype != LF_F32 && p->kernel != LF_KERNEL_SIMT;
   ws.qg_c = ws.ks_c = ws.vs_c = ws.part_acc = ws.part_ml = off;
   if (tc) {
-    ws.qg_c = off;
-    off = lf_align(off + B * H * Ga * LF_HD * eb);
-    ws.ks_c = off;
-    off = lf_align(off + B * H * Gka * LF_HD * eb);
-    ws.vs_c = off;
-    off = lf_align(off + B * H * Gka * LF_HD * eb);
     if (!for_bwd) {
-      // split-KV partials of the global rows
+      // split-KV partials of the global rows (the forward gathers the global
+      // tokens' rows itself)
       ws.part_acc = off;
       off = lf_align(off + B * H * Ga * dev.nch * LF_HD * 4);
       ws.part_ml = off;
       off = lf_align(off + B * H * Ga * dev.nch * 8);
     } else {
+      ws.qg_c = off;
+      off = lf_align(off + B * H * Ga * LF_HD * eb);
+      ws.ks_c = off;
+      off = lf_align(off + B * H * Gka * LF_HD * eb);
+      ws.vs_c = off;
+      off = lf_align(off + B * H * Gka * LF_HD * eb);
       // backward: per-chunk partials of the global columns (dK, dV) and rows (dQ_g)
       const size_t nchb = ((size_t)n + 63) / 64;  // rows per chunk of the global parts
       ws.part_acc = off;
@@ -208,8 +224,11 @@ static int lf_bind_ws(const lf_attn_params *p, int for_bwd, void *workspace, siz
   L.dev.binfo = (int32_t *)(L.ws_base + L.ws.binfo);
   L.dev.gidx = (int32_t *)(L.ws_base + L.ws.gidx);
   L.dev.grank = (int32_t *)(L.ws_base + L.ws.grank);
-  // each call starts with a clear status word; lf_attn_status reads it back
-  return lf_cuda(cudaMemsetAsync(L.dev.status, 0, LF_ST_WORDS * 4, L.stream), "status reset");
+  L.dev.wait_us = g_test_wait_us;
+  L.dev.skip_tile = g_test_skip_tile;
+  // each call starts with a clear status word (and split counters);
+  // lf_attn_status reads the word back
+  return lf_cuda(cudaMemsetAsync(L.dev.status, 0, L.ws.status_bytes, L.stream), "status reset");
 }
 
 extern "C" int lf_attn_fwd(const lf_attn_params *p, const void *q_s, const void *k_s,
@@ -226,21 +245,10 @@ extern "C" int lf_attn_fwd(const lf_attn_params *p, const void *q_s, const void 
   if ((st = lf_bind_ws(p, 0, workspace, ws_bytes, mask, stream, L))) return st;
   const bool tc = p->dtype != LF_F32 && p->kernel != LF_KERNEL_SIMT;
   if (tc) {
-    // the tensor-core path launches the mask pass itself (fused with its gather)
+    // the tensor-core path launches the mask pass itself; a shape outside its
+    // parameter block is refused (LF_ERR_UNSUPPORTED), never run elsewhere
     LfTcArgs a{q_s, k_s, v_s, q_g, k_g, v_g, o, lse, g_ev_start, g_ev_stop};
-    st = lf_tc_fwd(L, a, g_err, sizeof(g_err));
-    if (st == LF_ERR_UNSUPPORTED && p->kernel == LF_KERNEL_AUTO) {
-      // shape outside the tensor-core kernel's parameter block (refused before
-      // any launch): CUDA-core kernel
-      g_err[0] = 0;
-      st = LF_OK;
-      if ((st = lf_cuda(lf_launch_mask_pass(L), "mask pass"))) return st;
-      if (g_ev_start && g_ev_stop) cudaEventRecord(g_ev_start, L.stream);
-      if ((st = lf_cuda(lf_launch_simt_fwd(L, q_s, k_s, v_s, q_g, k_g, v_g, o, lse), "forward")))
-        return st;
-      if (g_ev_start && g_ev_stop) cudaEventRecord(g_ev_stop, L.stream);
-    }
-    if (st) return st;
+    if ((st = lf_tc_fwd(L, a, g_err, sizeof(g_err)))) return st;
   } else {
     if ((st = lf_cuda(lf_launch_mask_pass(L), "mask pass"))) return st;
     if (g_ev_start && g_ev_stop) cudaEventRecord(g_ev_start, L.stream);
@@ -271,9 +279,7 @@ extern "C" int lf_attn_bwd(const lf_attn_params *p, const void *q_s, const void 
   if ((st = lf_cuda(lf_launch_mask_pass(L), "mask pass"))) return st;
   if (p->dtype != LF_F32 && p->kernel != LF_KERNEL_SIMT) {
     LfTcBwdArgs a{q_s, k_s, v_s, q_g, k_g, v_g, o, lse, d_o, dq_s, dk_s, dv_s, dq_g, dk_g, dv_g};
-    st = lf_tc_bwd(L, a, g_err, sizeof(g_err));
-    if (st != LF_ERR_UNSUPPORTED || p->kernel != LF_KERNEL_AUTO) return st;
-    g_err[0] = 0;  // shape outside the tensor-core kernel's parameter block
+    return lf_tc_bwd(L, a, g_err, sizeof(g_err));  // refused shapes stay refused
   }
   return lf_cuda(lf_launch_simt_bwd(L, q_s, k_s, v_s, q_g, k_g, v_g, o, lse, d_o, dq_s, dk_s, dv_s,
                                     dq_g, dk_g, dv_g),

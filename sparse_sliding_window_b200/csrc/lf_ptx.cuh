@@ -48,10 +48,13 @@ __device__ __forceinline__ bool lf_mbar_try(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait on an mbarrier phase.  Returns false when the CTA aborted
-// (this thread's own timeout, or another role's).
+// (this thread's own timeout, or another role's).  abort_flag[0] is the
+// CTA's abort flag; abort_flag[1] the wait limit in microseconds (0: the
+// default LF_WAIT_NS), both in shared memory, set by the kernel at start.
 static __device__ __noinline__ bool lf_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                      int32_t *status, int site) {
   uint64_t t0 = 0;
+  const uint64_t limit = abort_flag[1] > 0 ? (uint64_t)abort_flag[1] * 1000ull : LF_WAIT_NS;
   for (uint32_t it = 0;; it++) {
     if (lf_mbar_try(bar, parity)) return true;
     if ((it & 255) == 255) {
@@ -59,8 +62,29 @@ static __device__ __noinline__ bool lf_wait(uint32_t bar, uint32_t parity, volat
       uint64_t now = lf_globaltimer();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > LF_WAIT_NS) {
+      } else if (now - t0 > limit) {
         *abort_flag = 1;
+        lf_set_status(status, LF_ERR_DEVICE_TIMEOUT, site);
+        return false;
+      }
+    }
+  }
+}
+
+// Wait for asynchronous work this CTA has already issued (TMA copies, MMAs)
+// to complete, also after an abort: the abort flag is not consulted, the
+// wait is bounded by time alone (LF_WAIT_NS); on expiry the status records
+// a timeout at `site`.
+static __device__ __noinline__ bool lf_wait_drain(uint32_t bar, uint32_t parity, int32_t *status,
+                                                  int site) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; it++) {
+    if (lf_mbar_try(bar, parity)) return true;
+    if ((it & 255) == 255) {
+      uint64_t now = lf_globaltimer();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > LF_WAIT_NS) {
         lf_set_status(status, LF_ERR_DEVICE_TIMEOUT, site);
         return false;
       }
@@ -242,6 +266,34 @@ __device__ __forceinline__ void lf_tmem_st32(uint32_t taddr, const float (&x)[32
       "r"(__float_as_uint(x[27])), "r"(__float_as_uint(x[28])), "r"(__float_as_uint(x[29])),
       "r"(__float_as_uint(x[30])), "r"(__float_as_uint(x[31]))
       : "memory");
+}
+
+// 8 consecutive fp32 columns of this thread's TMEM lane: load (waits) and store
+__device__ __forceinline__ void lf_tmem_ld8(uint32_t taddr, float (&x)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int k = 0; k < 8; k++) x[k] = __uint_as_float(r[k]);
+}
+__device__ __forceinline__ void lf_tmem_st8(uint32_t taddr, const float (&x)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+                   taddr),
+               "r"(__float_as_uint(x[0])), "r"(__float_as_uint(x[1])), "r"(__float_as_uint(x[2])),
+               "r"(__float_as_uint(x[3])), "r"(__float_as_uint(x[4])), "r"(__float_as_uint(x[5])),
+               "r"(__float_as_uint(x[6])), "r"(__float_as_uint(x[7]))
+               : "memory");
+}
+
+// 4 consecutive 32-bit columns of this thread's TMEM lane
+__device__ __forceinline__ void lf_tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c,
+                                            uint32_t d) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a),
+               "r"(b), "r"(c), "r"(d)
+               : "memory");
 }
 
 __device__ __forceinline__ void lf_tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {

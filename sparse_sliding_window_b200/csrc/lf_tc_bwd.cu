@@ -41,8 +41,8 @@
 
 #define LF_BW_THREADS 192
 #define LF_BW_NS 3
-#define LF_BW_MAX_MAPS 40
-#define LF_BW_MAX_SEG 32
+#define LF_BW_MAX_MAPS 192  // kernel parameters may take up to 32 KB
+#define LF_BW_MAX_SEG 96
 #define LF_BW_ROWS_PER_CHUNK 64  // rows (keys) per warp of the global-row / -column parts
 
 #define LF_BW_R0 0
@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
                  o_full = bar + 32, end_bar = bar + 40;
   const uint32_t col_full0 = bar + 48, col_empty0 = bar + 48 + 8 * LF_BW_NS;
   uint32_t *tmem_slot = (uint32_t *)(gbase + LF_BW_BAR + 192);
-  volatile int *abort_flag = (volatile int *)(gbase + LF_BW_BAR + 196);
+  volatile int *abort_flag = (volatile int *)(gbase + LF_BW_BAR + 196);  // [2]: flag, wait limit
 
   if (threadIdx.x == 0) {
     lf_mbar_init(row_full, 1);
@@ -147,7 +147,8 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
       lf_mbar_init(col_full0 + 8 * s, kModeQ ? 1 : 2);
       lf_mbar_init(col_empty0 + 8 * s, 1);
     }
-    *abort_flag = 0;
+    abort_flag[0] = 0;
+    abort_flag[1] = P.dev.wait_us;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
     }
     if (*abort_flag && lane == 0) {
       for (int t = max(0, issued - LF_BW_NS); t < issued; t++)
-        lf_wait(col_full0 + 8 * (t % LF_BW_NS), (t / LF_BW_NS) & 1, abort_flag, D.status, 22);
+        lf_wait_drain(col_full0 + 8 * (t % LF_BW_NS), (t / LF_BW_NS) & 1, D.status, 22);
     }
   } else if (warp == 5) {
     // ================================================== MMA issuer
@@ -278,7 +279,8 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
       }
     }
     lf_commit_w(end_bar);
-    lf_wait_warp(end_bar, 0, abort_flag, D.status, 27);
+    lf_wait_drain(end_bar, 0, D.status, 27);  // also after an abort: TMEM is freed after this
+    __syncwarp();
   } else {
     // ================================================== P / dS warps (0..3)
     const int q = warp * 32 + lane;
@@ -666,7 +668,9 @@ int lf_tc_bwd(const LfLaunch &L, const LfTcBwdArgs &a, char *err, size_t errlen)
       auto key = std::make_pair(d, rho);
       if (!rmap.count(key)) {
         if (nmaps + 4 > LF_BW_MAX_MAPS - 2) {
-          snprintf(err, errlen, "tensor-core backward: too many distinct dilation residues");
+          snprintf(err, errlen,
+                   "tensor-core backward: too many distinct dilation residues (the sum of the "
+                   "distinct dilations must stay <= %d)", (LF_BW_MAX_MAPS - 2) / 4);
           return LF_ERR_UNSUPPORTED;
         }
         const char *srcs[4] = {(const char *)a.qs, (const char *)a.ks, (const char *)a.vs,

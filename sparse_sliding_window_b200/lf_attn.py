@@ -24,7 +24,8 @@ ERROR_NAMES = {1: "LF_ERR_INVALID", 2: "LF_ERR_UNSUPPORTED", 3: "LF_ERR_CUDA",
 EXPORTS = ["lf_attn_version", "lf_attn_workspace_size", "lf_attn_fwd", "lf_attn_bwd",
            "lf_attn_count_pairs", "lf_attn_mask_dump", "lf_attn_status",
            "lf_attn_set_timing_events", "lf_attn_launch_count", "lf_attn_last_error",
-           "lf_attn_fwd_noalloc", "lf_attn_status_noalloc", "lf_attn_decode"]
+           "lf_attn_fwd_noalloc", "lf_attn_status_noalloc", "lf_attn_decode",
+           "lf_attn_set_test_hooks"]
 LF_STATIC_WORKSPACE_BYTES = 16 << 20
 
 
@@ -68,6 +69,8 @@ def load(path: str = LIB_PATH):
         lib.lf_attn_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         lib.lf_attn_decode.restype = i32
         lib.lf_attn_fwd_noalloc.restype = i32
+        lib.lf_attn_set_test_hooks.argtypes = [ctypes.c_uint32, i32]
+        lib.lf_attn_set_test_hooks.restype = i32
         lib.lf_attn_status_noalloc.argtypes = [vp]
         lib.lf_attn_status_noalloc.restype = i32
         for f in ("fwd", "bwd", "count_pairs", "mask_dump", "status", "set_timing_events"):
@@ -138,6 +141,11 @@ def lf_attn_fwd_noalloc(p, q_s, k_s, v_s, q_g, k_g, v_g, mask, o, lse, stream=No
     _check(load().lf_attn_fwd_noalloc(ctypes.byref(p), _ptr(q_s), _ptr(k_s), _ptr(v_s), _ptr(q_g),
                                       _ptr(k_g), _ptr(v_g), _ptr(mask), _ptr(o), _ptr(lse),
                                       _stream(stream)))
+
+
+def lf_attn_set_test_hooks(wait_limit_us: int = 0, skip_kv_tile: int = 0):
+    """Test hook of the device-side failure detection (see lf_attn.h)."""
+    _check(load().lf_attn_set_test_hooks(int(wait_limit_us), int(skip_kv_tile)))
 
 
 def lf_attn_status_noalloc(stream=None):

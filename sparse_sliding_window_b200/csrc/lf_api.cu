@@ -150,9 +150,7 @@ static int lf_prepare(const lf_attn_params *p, int for_bwd, LfDev &dev, LfWs &ws
   size_t off = 0;
   ws.status = off;
   {
-    size_t words = LF_ST_WORDS;
-    if (tc && !for_bwd) words += B * H * (((size_t)G + LF_BQ - 1) / LF_BQ);  // split counters
-    ws.status_bytes = words * 4;
+    ws.status_bytes = LF_ST_WORDS * 4;
     off = lf_align(off + ws.status_bytes);
   }
   ws.binfo = off;
@@ -163,20 +161,19 @@ static int lf_prepare(const lf_attn_params *p, int for_bwd, LfDev &dev, LfWs &ws
   off = lf_align(off + B * ((size_t)n + 1) * 4);
   ws.qg_c = ws.ks_c = ws.vs_c = ws.part_acc = ws.part_ml = off;
   if (tc) {
+    ws.qg_c = off;
+    off = lf_align(off + B * H * Ga * LF_HD * eb);
+    ws.ks_c = off;
+    off = lf_align(off + B * H * Gka * LF_HD * eb);
+    ws.vs_c = off;
+    off = lf_align(off + B * H * Gka * LF_HD * eb);
     if (!for_bwd) {
-      // split-KV partials of the global rows (the forward gathers the global
-      // tokens' rows itself)
+      // split-KV partials of the global rows
       ws.part_acc = off;
       off = lf_align(off + B * H * Ga * dev.nch * LF_HD * 4);
       ws.part_ml = off;
       off = lf_align(off + B * H * Ga * dev.nch * 8);
     } else {
-      ws.qg_c = off;
-      off = lf_align(off + B * H * Ga * LF_HD * eb);
-      ws.ks_c = off;
-      off = lf_align(off + B * H * Gka * LF_HD * eb);
-      ws.vs_c = off;
-      off = lf_align(off + B * H * Gka * LF_HD * eb);
       // backward: per-chunk partials of the global columns (dK, dV) and rows (dQ_g)
       const size_t nchb = ((size_t)n + 63) / 64;  // rows per chunk of the global parts
       ws.part_acc = off;

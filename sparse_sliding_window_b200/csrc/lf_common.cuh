@@ -32,15 +32,14 @@
 // Workspace carve-up (byte offsets, each 256-byte aligned); computed on the
 // host from the params, passed to every kernel.
 struct LfWs {
-  size_t status;    // int32[LF_ST_WORDS], then (tensor-core forward) int32[B][H][ceil(G/128)]
-                    // counters of the split partials written per global row group
+  size_t status;    // int32[LF_ST_WORDS]
   size_t status_bytes;  // bytes of the status block, zeroed at the start of every call
   size_t binfo;     // int32[B][LF_BI_WORDS]
   size_t gidx;      // int32[B][G]           global positions, ascending
   size_t grank;     // int32[B][n+1]         globals at positions < p
-  size_t qg_c;      // T[B][H][G][64]        backward: Q_g rows of the global tokens
-  size_t ks_c;      // T[B][H][Gk][64]       backward: K_s rows of the global tokens (zero padded)
-  size_t vs_c;      // T[B][H][Gk][64]       backward: V_s rows of the global tokens (zero padded)
+  size_t qg_c;      // T[B][H][G][64]        Q_g rows of the global tokens
+  size_t ks_c;      // T[B][H][Gk][64]       K_s rows of the global tokens (zero padded)
+  size_t vs_c;      // T[B][H][Gk][64]       V_s rows of the global tokens (zero padded)
   size_t part_acc;  // float[B][H][G][NCH][64] split-KV partial sums of global rows
   size_t part_ml;   // float2[B][H][G][NCH]   (running max, running sum) of each split
   size_t delta;     // float[B][H][n]        backward: rowsum(dO * O)

@@ -236,15 +236,16 @@ __device__ __forceinline__ void lf_tmem_ld32(uint32_t taddr, float (&x)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
       "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
+      "%28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
         "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
         "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      : "r"(taddr)
+      : "memory");
 #pragma unroll
   for (int k = 0; k < 32; k++) x[k] = __uint_as_float(r[k]);
 }
@@ -271,11 +272,12 @@ __device__ __forceinline__ void lf_tmem_st32(uint32_t taddr, const float (&x)[32
 // 8 consecutive fp32 columns of this thread's TMEM lane: load (waits) and store
 __device__ __forceinline__ void lf_tmem_ld8(uint32_t taddr, float (&x)[8]) {
   uint32_t r[8];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+               "tcgen05.wait::ld.sync.aligned;"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
                  "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+               : "r"(taddr)
+               : "memory");
 #pragma unroll
   for (int k = 0; k < 8; k++) x[k] = __uint_as_float(r[k]);
 }
@@ -303,6 +305,20 @@ __device__ __forceinline__ void lf_tmem_st16(uint32_t taddr, const uint32_t (&w)
       "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
       "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]),
       "r"(w[15])
+      : "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane; the load and
+// its wait are one statement, so no use of r can move above the wait
+__device__ __forceinline__ void lf_tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
       : "memory");
 }
 
@@ -364,11 +380,6 @@ __device__ __forceinline__ int lf_reg(int x) {
   return y;
 }
 
-// One pass over the 4 column chunks of a row's S tile (TMEM lane of this
-// thread).  Columns whose bit in w is clear are treated as -inf.  Tracks the
-// row max of the attended raw scores in mx; when write_p, also computes
-// p = 2^(s * sl2 - m) into P (TMEM, packed bf16 / f16) and their sum lt.
-// Chunks no lane of the warp attends are skipped (P written as zeros).
 // TMEM load of 32 columns without waiting; the caller waits with
 // lf_tmem_wait_ld_regs, which also pins the registers behind the wait.
 __device__ __forceinline__ void lf_tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {

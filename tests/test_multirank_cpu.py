@@ -45,7 +45,7 @@ def _worker(rank, world, port, results):
 def test_two_rank_max_and_job_throughput():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of a multi-threaded process
     results = mgr.dict()
     mp.spawn(_worker, args=(world, port, results), nprocs=world, join=True)
     for r in range(world):

@@ -58,6 +58,10 @@ def _cases():
     C["n1"] = dict(B=1, H=1, n=1, r=4, dil=[1], causal=False, mask=_mask(1, 1))
     # a causal window wider than the sequence: full causal (decoder) self-attention
     C["causal_dense"] = dict(B=1, H=2, n=600, r=1000, dil=[1, 1], causal=True, mask=_mask(1, 600))
+    # 11 residue sub-sequences (1 + 2 + 8): more tensor maps than a small
+    # parameter block holds; the tensor-core kernels take it (no fallback)
+    C["dil_1_2_8"] = dict(B=1, H=3, n=1100, r=40, dil=[1, 2, 8], causal=False,
+                          mask=_mask(1, 1100, globals_=[[0, 555]]))
     # large scores (inputs N(0, 3^2) / N(0, 4^2)): row sums leave the range the
     # running reference allows, so the tensor-core softmax redoes tiles with
     # the row's tile max (overflow side) and, with two keys per row, with
@@ -140,11 +144,12 @@ def test_pair_counts_and_pattern_exact(name):
             assert np.array_equal(dump[b, h], A), (b, h)
 
 
-# The large-score cases exercise the forward's running-reference redo; the
-# backward has no such logic (P comes from the saved lse), and with nearly
-# one-hot rows its error is set by the cancellation in dP - D, outside the
-# unit-scale tolerance derivation, so it runs on the unit-scale cases only.
+# Unit-scale cases take the fixed bounds below.  On the large-score cases
+# (nearly one-hot rows) the 16-bit error is set by the cancellation in
+# dS = p (dP - D) and scales with the inputs; those take the elementwise
+# first-order bound of lfutil.bwd_error_bound instead (test below).
 BWD_CASES = sorted(k for k, c in CASES.items() if c.get("in_scale", 1.0) == 1.0)
+HOT_CASES = sorted(k for k, c in CASES.items() if c.get("in_scale", 1.0) != 1.0)
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
@@ -159,6 +164,49 @@ def test_backward_parity(name, dtype):
     # the oracle sees the same rounded dO
     ref = oracle.bwd(c["r"], c["dil"], c["causal"], U.scale_of(wl), inp["mask"], f["qs"], f["ks"],
                      f["vs"], f["qg"], f["kg"], f["vg"], f["do"])
+    for k, nm in enumerate(["dq_s", "dk_s", "dv_s", "dq_g", "dk_g", "dv_g"]):
+        U.compare(name + "/" + nm, U.to_f64(grads[k]), ref[k], dtype)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("name", HOT_CASES)
+def test_backward_parity_large_scores(name, dtype):
+    """Backward on Q, K at 3x / 4x scale: every gradient element within the
+    derived first-order bound (dS and P rounded to the format, D from the
+    rounded forward output) plus the rounding of the stored gradient."""
+    c, wl, inp, att = _setup(name, dtype, L.LF_KERNEL_TC, backward=True)
+    g = U.gpu_inputs(inp, dtype)
+    o, lse = att.fwd(g["qs"], g["ks"], g["vs"], g["qg"], g["kg"], g["vg"], g["mask"])
+    grads = att.bwd(g["qs"], g["ks"], g["vs"], g["qg"], g["kg"], g["vg"], g["mask"], o, lse, g["do"])
+    att.status(bwd=True)
+    f = U.f64_inputs(inp, dtype)
+    scale = U.scale_of(wl)
+    ref = oracle.bwd(c["r"], c["dil"], c["causal"], scale, inp["mask"], f["qs"], f["ks"], f["vs"],
+                     f["qg"], f["kg"], f["vg"], f["do"])
+    bound = U.bwd_error_bound(c, scale, inp["mask"], f, dtype)
+    for k, nm in enumerate(["dq_s", "dk_s", "dv_s", "dq_g", "dk_g", "dv_g"]):
+        U.compare_bound(name + "/" + nm, U.to_f64(grads[k]), ref[k], bound[k], dtype, factor=1.0)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_tensor_core_many_residues_fwd_bwd(dtype):
+    """Dilations 1, 2, 8 on the tensor-core kernels, asked for explicitly:
+    both run it (the shape is inside their parameter blocks) and match."""
+    name = "dil_1_2_8"
+    c, wl, inp, att = _setup(name, dtype, L.LF_KERNEL_TC, backward=True)
+    g = U.gpu_inputs(inp, dtype)
+    o, lse = att.fwd(g["qs"], g["ks"], g["vs"], g["qg"], g["kg"], g["vg"], g["mask"])
+    att.status()
+    grads = att.bwd(g["qs"], g["ks"], g["vs"], g["qg"], g["kg"], g["vg"], g["mask"], o, lse, g["do"])
+    att.status(bwd=True)
+    f = U.f64_inputs(inp, dtype)
+    scale = U.scale_of(wl)
+    ro, rl = oracle.fwd(c["r"], c["dil"], c["causal"], scale, inp["mask"], f["qs"], f["ks"], f["vs"],
+                        f["qg"], f["kg"], f["vg"])
+    U.compare(name + "/o", U.to_f64(o), ro, dtype)
+    U.compare_lse(U.to_f64(lse), rl, dtype)
+    ref = oracle.bwd(c["r"], c["dil"], c["causal"], scale, inp["mask"], f["qs"], f["ks"], f["vs"],
+                     f["qg"], f["kg"], f["vg"], f["do"])
     for k, nm in enumerate(["dq_s", "dk_s", "dv_s", "dq_g", "dk_g", "dv_g"]):
         U.compare(name + "/" + nm, U.to_f64(grads[k]), ref[k], dtype)
 

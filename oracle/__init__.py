@@ -57,7 +57,8 @@ def _load():
         lib.lf_oracle_probs_row.argtypes = [i32, i32, i32, i32, i32, dbl, p, p, p, p, p, i32, p]
         lib.lf_oracle_fwd_head.argtypes = [i32, i32, i32, i32, i32, dbl, p] + [p] * 6 + [p, p]
         lib.lf_oracle_bwd_head.argtypes = [i32, i32, i32, i32, i32, dbl, p] + [p] * 7 + [p] * 6
-        for f in ("pattern", "count_pairs", "probs_row", "fwd_head", "bwd_head"):
+        lib.lf_oracle_linear.argtypes = [i32, i32, i32, p, p, p, p]
+        for f in ("pattern", "count_pairs", "probs_row", "fwd_head", "bwd_head", "linear"):
             getattr(lib, "lf_oracle_" + f).restype = i32
         _lib = lib
     return _lib
@@ -180,3 +181,22 @@ def counts(r: int, dilation, causal: bool, mask, H: int) -> np.ndarray:
                 cache[key] = count_pairs(n, r, int(dilation[h]), causal, mask[b])
             out[b, h] = cache[key]
     return out
+
+
+def linear(x, w, b=None) -> np.ndarray:
+    """The affine map y = x w^T + b over the last axis of x (float64), with
+    w in the [out_features, in_features] layout: the projections into
+    Qs/Ks/Vs/Qg/Kg/Vg and the output projection around the attention."""
+    x = _f64(x)
+    w = _f64(w)
+    N, K = w.shape
+    assert x.shape[-1] == K
+    lead = x.shape[:-1]
+    M = int(np.prod(lead)) if lead else 1
+    xb = np.ascontiguousarray(x.reshape(M, K))
+    bb = None if b is None else _f64(b)
+    assert bb is None or bb.shape == (N,)
+    y = np.zeros((M, N), dtype=np.float64)
+    _check(_load().lf_oracle_linear(M, N, K, _ptr(xb), _ptr(w), None if bb is None else _ptr(bb), _ptr(y)))
+    return y.reshape(lead + (N,))
+

@@ -346,3 +346,29 @@ int lf_oracle_bwd_head(int n, int hd, int r, int d, int causal, double scale,
   orc_pattern_free(&A);
   return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------
+ * The linear projections either side of the attention (segmentfault page,
+ * section 全局注意力的线性投影: the hidden states are projected by separate
+ * linear maps into Qs, Ks, Vs and Qg, Kg, Vg).  An affine map in the
+ * [out_features, in_features] weight layout:
+ *
+ *   y[m][c] = sum_k x[m][k] * w[c][k] + b[c]        (b may be NULL)
+ *
+ * computed in double, one output element at a time, rows in parallel.
+ * ------------------------------------------------------------------------ */
+int lf_oracle_linear(int M, int N, int K, const double *x, const double *w, const double *b,
+                     double *y) {
+  if (M < 0 || N < 0 || K < 0 || !x || !w || !y) return ORC_ERR_ARG;
+#pragma omp parallel for schedule(static)
+  for (int m = 0; m < M; m++) {
+    const double *xr = x + (size_t)m * K;
+    for (int c = 0; c < N; c++) {
+      const double *wr = w + (size_t)c * K;
+      double s = 0.0;
+      for (int k = 0; k < K; k++) s += xr[k] * wr[k];
+      y[(size_t)m * N + c] = s + (b ? b[c] : 0.0);
+    }
+  }
+  return ORC_OK;
+}

@@ -32,6 +32,9 @@ MUTANTS = {
     "bwd_delta_dropped": ("double ds = p * (orc_dot(g, vj, hd) - delta[i]);", "double ds = p * orc_dot(g, vj, hd);"),
     "bwd_dv_wrong_weight": ("dv[c] += p * g[c];", "dv[c] += ds * g[c];"),
     "bwd_dk_transposed": ("dk[c] += scale * ds * q[c];", "dk[c] += scale * ds * kj[c];"),
+    "linear_weight_transposed": ("for (int k = 0; k < K; k++) s += xr[k] * wr[k];",
+                                 "for (int k = 0; k < K; k++) s += xr[k] * w[(size_t)k * N + c];"),
+    "linear_bias_dropped": ("y[(size_t)m * N + c] = s + (b ? b[c] : 0.0);", "y[(size_t)m * N + c] = s;"),
     "bwd_dq_unscaled": ("for (int c = 0; c < hd; c++) dq[c] += scale * ds * kj[c];",
                         "for (int c = 0; c < hd; c++) dq[c] += ds * kj[c];"),
 }
@@ -52,6 +55,7 @@ def _pins():
         (pins.test_backward_finite_differences, ("band_global_pad",)),
         (pins.test_backward_finite_differences, ("dilated",)),
         (pins.test_backward_zero_rows, ()),
+        (pins.test_linear_matches_numpy_and_special_cases, ()),
     ]
 
 
@@ -68,7 +72,7 @@ def test_mutant_is_caught(name, monkeypatch):
         subprocess.check_call(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", so, c, "-lm"])
         real = oracle._load()
         lib = ctypes.CDLL(so)
-        for f in ("threads", "pattern", "count_pairs", "probs_row", "fwd_head", "bwd_head"):
+        for f in ("threads", "pattern", "count_pairs", "probs_row", "fwd_head", "bwd_head", "linear"):
             fn = getattr(lib, "lf_oracle_" + f)
             ref = getattr(real, "lf_oracle_" + f)
             fn.restype = ref.restype

@@ -299,3 +299,25 @@ def test_workload_masks():
         assert m[b, 0] == 2 and int((m[b] == 2).sum()) == 17
     m = synth.build_mask(synth.WORKLOADS["base_bf16"])
     assert (m[0, :65] == 2).all() and (m[0, 65:] == 1).all()
+
+
+# ---------------------------------------------------------------- projections
+
+def test_linear_matches_numpy_and_special_cases():
+    """oracle.linear (the projections either side of the attention) against
+    numpy's matmul on non-square, non-symmetric shapes, and against what the
+    definition fixes: an identity weight copies x, a zero input gives the
+    bias, and the map is linear in x without the bias."""
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((3, 5, 6))
+    w = rng.standard_normal((4, 6))
+    b = rng.standard_normal(4)
+    np.testing.assert_allclose(oracle.linear(x, w, b), x @ w.T + b, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(oracle.linear(x, w), x @ w.T, rtol=0, atol=1e-12)
+    sq = rng.standard_normal((6, 6))  # square, non-symmetric: a transposed index shows
+    np.testing.assert_allclose(oracle.linear(x, sq), x @ sq.T, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(oracle.linear(x, np.eye(6)), x)
+    np.testing.assert_array_equal(oracle.linear(np.zeros((2, 6)), w, b), np.tile(b, (2, 1)))
+    x2 = rng.standard_normal((3, 5, 6))
+    np.testing.assert_allclose(oracle.linear(2.5 * x + x2, w), 2.5 * oracle.linear(x, w) + oracle.linear(x2, w),
+                               rtol=0, atol=1e-12)

@@ -368,6 +368,73 @@ def decode_numbers(wl, steps, warmup, dev):
                          "note": "CUDA-graph replay of 32 steps; a step still includes the device-side launch gap"}}
 
 
+def projection_numbers(wl, steps, warmup, dev):
+    """The projections around one attention layer of the workload's shape,
+    each GEMM timed by CUDA events the library records around its kernel,
+    with L2 flushed (a 256 MB write) before every timed call:
+      in:  hidden [B, n, d_model] -> Q_s, K_s, V_s, K_g, V_g (one call, N = 5 d_model)
+      qg:  Q_g at the sequence's global tokens only (row gather + GEMM)
+      out: heads [B, H, n, 64] -> [B, n, d_model]
+    FLOPs are 2 M N K of the rows computed."""
+    import torch
+    from sparse_sliding_window_b200 import lf_attn as L
+    B, n, H = wl.B, wl.n, wl.H
+    D = H * wl.head_dim
+    tdt = torch.float16 if wl.dtype == "f16" else torch.bfloat16
+    g = torch.Generator(device=dev).manual_seed(1234)
+
+    def rnd(*shape, scale=1.0):
+        return (torch.randn(*shape, device=dev, generator=g) * scale).to(tdt)
+
+    x = rnd(B, n, D)
+    w_in, b_in = rnd(5 * D, D, scale=D ** -0.5), rnd(5 * D, scale=0.1)
+    w_qg, b_qg = rnd(D, D, scale=D ** -0.5), rnd(D, scale=0.1)
+    w_out, b_out = rnd(D, D, scale=D ** -0.5), rnd(D, scale=0.1)
+    o = rnd(B, H, n, wl.head_dim)
+    outs = [torch.empty(B, H, n, wl.head_dim, device=dev, dtype=tdt) for _ in range(6)]
+    y = torch.empty(B, n, D, device=dev, dtype=tdt)
+    mask = torch.from_numpy(synth.build_mask(wl)).to(dev)
+    ng = int((mask == 2).sum(dim=1).max().item())
+    p = L.make_proj_params(B, n, H, L.LF_BF16 if wl.dtype != "f16" else L.LF_F16)
+    ws = L.proj_workspace(p, max(ng, 1))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    calls = {
+        "in": (lambda: L.lf_proj_in(p, x, w_in, b_in, outs[:5], ws), 2.0 * B * n * 5 * D * D),
+        "out": (lambda: L.lf_proj_out(p, o, w_out, b_out, y, ws), 2.0 * B * n * D * D),
+    }
+    if ng > 0:
+        calls["qg"] = (lambda: L.lf_proj_in(p, x, w_qg, b_qg, outs[5:], ws, rows_mask=mask,
+                                            rows_code=2, max_rows=ng),
+                       2.0 * int((mask == 2).sum().item()) * D * D)
+    a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    c.record()
+    pk = _peaks()
+    res = {}
+    for name, (fn, flops) in calls.items():
+        for _ in range(max(3, warmup)):
+            fn()
+        torch.cuda.synchronize(dev)
+        ts = []
+        for _ in range(max(5, min(steps, 50))):
+            flush.zero_()
+            L.lf_proj_set_timing_events(a, c)
+            fn()
+            L.lf_proj_set_timing_events(None, None)
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(c) * 1e-3)
+        L.lf_attn_status(ws)
+        ts.sort()
+        t = ts[len(ts) // 2]
+        res[name] = {"kernel_us": t * 1e6, "tflops": flops / t * 1e-12,
+                     "frac": flops / t * 1e-12 / pk["bf16"], "flops": flops}
+    res["peak_tflops"] = pk["bf16"]
+    res["peak_source"] = pk["src"]
+    res["shape"] = {"B": B, "n": n, "d_model": D, "heads": H, "global_rows": int((mask == 2).sum().item())}
+    res["timing"] = "median over calls, CUDA events around each GEMM kernel, L2 flushed before each"
+    return res
+
+
 def run_decode(args, wl):
     import torch
     dev = torch.device("cuda", 0)
@@ -583,6 +650,8 @@ def main():
                     help="also time the backward (default for workloads with a backward)")
     ap.add_argument("--no-others", action="store_true",
                     help="skip the other workloads reported under 'workloads'")
+    ap.add_argument("--proj", action="store_true",
+                    help="time only the projection GEMMs around the layer (one JSON line)")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
     layout = resolve_world(args.gpus)
@@ -597,6 +666,17 @@ def main():
 
     if args.decode:
         return run_decode(args, wl)
+    if args.proj:
+        pr = projection_numbers(wl, args.steps, args.warmup, torch.device("cuda", 0))
+        tot_f = sum(v["flops"] for k, v in pr.items() if isinstance(v, dict) and "flops" in v)
+        tot_t = sum(v["kernel_us"] for k, v in pr.items() if isinstance(v, dict) and "flops" in v)
+        print(json.dumps({"metric": "projection GEMM TFLOP/s (input, global-row and output projections)",
+                          "value": tot_f / tot_t * 1e-6, "unit": "TFLOP/s", "n_gpus": 1,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t * 1e-3,
+                          "higher_is_better": True, "dtype": wl.dtype, "data": "synthetic",
+                          "config": {"workload": wl.name + " projections"}, "projections": pr}),
+              flush=True)
+        return 0
     world, rank, local = layout
     if world > 1:
         import datetime
@@ -632,6 +712,8 @@ def main():
         line["backward"] = time_backward(m["att"], m["sets"][0], wl, pairs, world, args.steps,
                                          args.warmup, dev, stream)
     del m
+    if world == 1 and args.kernel != "simt":
+        line["projections"] = projection_numbers(wl, args.steps, args.warmup, dev)
     if not args.no_others and args.kernel != "simt":
         # every other workload, driver-observed beside the headline: its
         # forward step / main kernel / roofline, the backward where it has

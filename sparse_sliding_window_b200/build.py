@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "liblf_attn.so")
-SOURCES = ["lf_api.cu", "lf_simt.cu", "lf_tc.cu", "lf_tc_bwd.cu", "lf_static.cu"]
+SOURCES = ["lf_api.cu", "lf_simt.cu", "lf_tc.cu", "lf_tc_bwd.cu", "lf_static.cu", "lf_gemm.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -28,7 +28,7 @@ def needs_build() -> bool:
         return True
     t = os.path.getmtime(LIB)
     deps = sources() + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")]
-    deps.append(os.path.join(ROOT, "include", "lf_attn.h"))
+    deps += [os.path.join(ROOT, "include", h) for h in ("lf_attn.h", "lf_proj.h")]
     return any(os.path.getmtime(s) > t for s in deps)
 
 

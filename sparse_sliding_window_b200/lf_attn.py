@@ -26,6 +26,8 @@ EXPORTS = ["lf_attn_version", "lf_attn_workspace_size", "lf_attn_fwd", "lf_attn_
            "lf_attn_set_timing_events", "lf_attn_launch_count", "lf_attn_last_error",
            "lf_attn_fwd_noalloc", "lf_attn_status_noalloc", "lf_attn_decode",
            "lf_attn_set_test_hooks"]
+# every symbol include/lf_proj.h declares
+PROJ_EXPORTS = ["lf_proj_workspace_size", "lf_proj_in", "lf_proj_out", "lf_proj_set_timing_events"]
 LF_STATIC_WORKSPACE_BYTES = 16 << 20
 
 
@@ -41,6 +43,11 @@ class lf_attn_params(ctypes.Structure):
                 ("dilation", ctypes.POINTER(ctypes.c_int32)), ("causal", ctypes.c_int),
                 ("scale", ctypes.c_float), ("dtype", ctypes.c_int), ("max_global", ctypes.c_int),
                 ("kernel", ctypes.c_int)]
+
+
+class lf_proj_params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("n", ctypes.c_int), ("H", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("dtype", ctypes.c_int)]
 
 
 _lib = None
@@ -75,6 +82,15 @@ def load(path: str = LIB_PATH):
         lib.lf_attn_status_noalloc.restype = i32
         for f in ("fwd", "bwd", "count_pairs", "mask_dump", "status", "set_timing_events"):
             getattr(lib, "lf_attn_" + f).restype = i32
+        PP = ctypes.POINTER(lf_proj_params)
+        lib.lf_proj_workspace_size.argtypes = [PP, i32]
+        lib.lf_proj_workspace_size.restype = sz
+        lib.lf_proj_in.argtypes = [PP, i32, vp, vp, vp, ctypes.POINTER(vp), vp, i32, i32, vp, sz, vp]
+        lib.lf_proj_in.restype = i32
+        lib.lf_proj_out.argtypes = [PP, vp, vp, vp, vp, vp, sz, vp]
+        lib.lf_proj_out.restype = i32
+        lib.lf_proj_set_timing_events.argtypes = [vp, vp]
+        lib.lf_proj_set_timing_events.restype = i32
         _lib = lib
     return _lib
 
@@ -191,6 +207,47 @@ def lf_attn_set_timing_events(ev_start, ev_stop):
 
 def lf_attn_launch_count() -> int:
     return int(load().lf_attn_launch_count())
+
+
+def make_proj_params(B: int, n: int, H: int, dtype: int = LF_BF16, head_dim: int = 64):
+    p = lf_proj_params()
+    p.B, p.n, p.H, p.head_dim, p.dtype = B, n, H, head_dim, dtype
+    return p
+
+
+def lf_proj_workspace_size(p, max_rows: int = 0) -> int:
+    return int(load().lf_proj_workspace_size(ctypes.byref(p), int(max_rows)))
+
+
+def proj_workspace(p, max_rows: int = 0, device="cuda"):
+    """Allocate a projection workspace (a uint8 torch tensor, 256-B aligned)."""
+    import torch
+    nbytes = lf_proj_workspace_size(p, max_rows)
+    if nbytes == 0:
+        _check(LF_ERR_INVALID)
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def lf_proj_in(p, x, w_in, b_in, outs, ws, rows_mask=None, rows_code: int = 2, max_rows: int = 0,
+               stream=None):
+    """Input projections: outs[k][b,h,t,:] = x[b,t,:] . w_in[k*D + h*64 + :, :] + b_in[...]
+    (only rows with rows_mask == rows_code when a mask is given)."""
+    arr = (ctypes.c_void_p * len(outs))(*[o.data_ptr() for o in outs])
+    _check(load().lf_proj_in(ctypes.byref(p), len(outs), _ptr(x), _ptr(w_in), _ptr(b_in), arr,
+                             _ptr(rows_mask), int(rows_code), int(max_rows), _ptr(ws), ws.numel(),
+                             _stream(stream)))
+
+
+def lf_proj_out(p, o, w_out, b_out, y, ws, stream=None):
+    """Output projection: y[b,t,:] = concat_h o[b,h,t,:] . w_out^T + b_out."""
+    _check(load().lf_proj_out(ctypes.byref(p), _ptr(o), _ptr(w_out), _ptr(b_out), _ptr(y), _ptr(ws),
+                              ws.numel(), _stream(stream)))
+
+
+def lf_proj_set_timing_events(ev_start, ev_stop):
+    a = None if ev_start is None else ev_start.cuda_event
+    b = None if ev_stop is None else ev_stop.cuda_event
+    _check(load().lf_proj_set_timing_events(a, b))
 
 
 # ------------------------------------------------------------ convenience --

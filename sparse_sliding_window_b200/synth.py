@@ -38,7 +38,10 @@ _M2 = np.uint64(0x94D049BB133111EB)
 
 # stream ids of the tensors a workload draws
 STREAMS = {"qs": 1, "ks": 2, "vs": 3, "qg": 4, "kg": 5, "vg": 6, "do": 7,
-           "lengths": 8, "globals": 9}
+           "lengths": 8, "globals": 9,
+           # the projections around the attention: hidden states, input
+           # weights and biases, attention output, output weights and bias
+           "x": 10, "w": 11, "b": 12, "o": 13, "wo": 14, "bo": 15}
 
 
 def _mix(z: np.ndarray) -> np.ndarray:

@@ -96,3 +96,36 @@ def test_decode_host_validation_without_gpu(lib):
     assert rc == L.LF_ERR_INVALID and b"q" in lib.lf_attn_last_error()
     rc = lib.lf_attn_decode(ctypes.byref(pc), vp(a16), vp(a16 + 4), *([vp(a16)] * 3), None, None)
     assert rc == L.LF_ERR_INVALID and b"aligned" in lib.lf_attn_last_error()
+
+
+def test_projection_abi_exports_and_host_checks(lib):
+    """include/lf_proj.h: every declared symbol is exported and bound, the
+    workspace is sized, and bad arguments are refused on the host."""
+    text = open(os.path.join(ROOT, "include", "lf_proj.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = sorted(set(re.findall(r"\b(lf_proj_\w+)\s*\(", text)))
+    assert names == sorted(L.PROJ_EXPORTS)
+    for name in names:
+        assert hasattr(lib, name), name
+    p = L.make_proj_params(2, 4096, 12, L.LF_BF16)
+    w0 = L.lf_proj_workspace_size(p, 0)
+    w1 = L.lf_proj_workspace_size(p, 65)
+    assert 0 < w0 < w1 and w0 % 256 == 0 and w1 % 256 == 0
+    assert w1 >= 2 * 65 * 768 * 2  # the gathered rows' hidden states
+    for bad in (dict(B=0), dict(n=0), dict(H=6), dict(H=0), dict(dtype=L.LF_F32), dict(head_dim=32)):
+        kw = dict(B=1, n=128, H=12, dtype=L.LF_BF16)
+        kw.update(bad)
+        hd = kw.pop("head_dim", 64)
+        assert L.lf_proj_workspace_size(L.make_proj_params(head_dim=hd, **kw), 0) == 0, bad
+    buf = (ctypes.c_char * 8192)()
+    a = (ctypes.addressof(buf) + 255) & ~255
+    outs = (ctypes.c_void_p * 1)(a)
+    q = L.make_proj_params(1, 128, 12, L.LF_BF16)
+    # NULL x, misaligned weight, nproj out of range, workspace too small: no launch
+    assert lib.lf_proj_in(ctypes.byref(q), 1, None, a, None, outs, None, 2, 0, a, 4096, None) == L.LF_ERR_INVALID
+    assert lib.lf_proj_in(ctypes.byref(q), 1, a, a + 2, None, outs, None, 2, 0, a, 4096, None) == L.LF_ERR_INVALID
+    assert lib.lf_proj_in(ctypes.byref(q), 9, a, a, None, outs, None, 2, 0, a, 4096, None) == L.LF_ERR_INVALID
+    assert lib.lf_proj_in(ctypes.byref(q), 1, a, a, None, outs, a, 2, 0, a, 4096, None) == L.LF_ERR_INVALID
+    assert lib.lf_proj_out(ctypes.byref(q), a, a, None, a, a, 16, None) == L.LF_ERR_INVALID
+    assert lib.lf_proj_out(ctypes.byref(L.make_proj_params(1, 128, 6, L.LF_BF16)), a, a, None, a, a,
+                           4096, None) == L.LF_ERR_UNSUPPORTED

@@ -14,15 +14,18 @@
 //     concatenated by the loads themselves; plain [B, n, d_model] out.
 //
 // Persistent, one CTA of 192 threads per SM, output tiles of 128 rows x 256
-// features, the reduction in k-steps of 64:
+// features (128 when 256-wide tiles would leave SMs idle), the reduction in
+// k-steps of 64:
 //   warp 0  TMA producer: per k-step a 128x64 tile of A and a 256x64 tile of
 //           W (128-byte swizzle, K-major) into a 4-stage ring (48 KB each)
 //   warp 1  MMA issuer (owns TMEM): four K = 16 tcgen05.mma (M = 128,
 //           N = 256) per k-step into one of two 256-column fp32 accumulators
-//   warps 2-5  epilogue: TMEM -> registers (32 columns at a time, the next
-//           chunk loading while this one is stored) -> + bias -> dtype ->
-//           global memory; frees the accumulator for the tile after next,
-//           so the epilogue of one tile overlaps the main loop of the next.
+//   warps 2-5  epilogue: per 64-column box, TMEM -> registers -> + bias ->
+//           dtype -> shared memory in the 128-byte swizzle layout -> one TMA
+//           store (two staging boxes alternate); it frees the accumulator for
+//           the tile after next, so the epilogue of one tile overlaps the
+//           main loop of the next.  Gathered rows (Q_g) are scattered to their
+//           positions with plain stores instead.
 // Tiles go row-block-major, feature-block fastest, so the CTAs running at
 // one time share their A tiles in L2.  No TMA multicast is used.
 //
@@ -43,23 +46,29 @@
 #include "lf_tc.cuh"
 
 #define LG_BM 128
-#define LG_BN 256
 #define LG_BK 64
 #define LG_NS 4
 #define LG_THREADS 192
 #define LG_A_BYTES (LG_BM * LG_BK * 2)
-#define LG_B_BYTES (LG_BN * LG_BK * 2)
-#define LG_STAGE (LG_A_BYTES + LG_B_BYTES)
-#define LG_BAR (LG_NS * LG_STAGE)
-#define LG_SMEM (LG_BAR + 1024)
 #define LG_MAX_OUT 8
-static_assert(LG_SMEM <= 232448, "shared memory per CTA");
+// per output-tile width kBN (256, or 128 when the 256-wide tiles would leave
+// SMs idle): stage = A tile + W tile; then two 128 x 64 output staging boxes
+// (16 KB each) and the barriers
+template <int kBN> struct LgLayout {
+  static constexpr int B_BYTES = kBN * LG_BK * 2;
+  static constexpr int STAGE = LG_A_BYTES + B_BYTES;
+  static constexpr int STG = LG_NS * STAGE;
+  static constexpr int BAR = STG + 2 * LG_BM * 64 * 2;
+  static constexpr int SMEM = BAR + 1024;
+  static_assert(SMEM <= 232448, "shared memory per CTA");
+};
 
 int lf_record_error(int code, const char *msg);
 
 struct LgParams {
   CUtensorMap map_a;  // mode 0: {K, L, B} box {64, 128, 1}; mode 1: {64, L, H, B} box {64, 128, 1, 1}
   CUtensorMap map_b;  // W [N, K]: {K, N} box {64, 256}
+  CUtensorMap map_out[LG_MAX_OUT];  // stores: head split {64, Lout, H, B} / plain {N, L, B}, box 64 x 128
   int mode;           // 0: A rows of K elements; 1: A = heads [B, H, L, 64], k-step = head
   int B, L, K, N;     // L: rows of A per sequence
   int ksteps, mblk, nblk, tiles;
@@ -102,6 +111,21 @@ __device__ __forceinline__ void lg_tma2(uint32_t dst, const CUtensorMap *map, ui
       : "memory");
 }
 
+// TMA stores of one 128-row x 64-column box from shared memory (bulk group)
+__device__ __forceinline__ void lg_store4(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2,
+                                          int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void lg_store3(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(src)
+               : "memory");
+}
+
 __device__ __forceinline__ void lg_tma3(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0,
                                         int c1, int c2) {
   asm volatile(
@@ -123,8 +147,9 @@ __device__ __forceinline__ LgTile lg_tile(const LgParams &P, int tile) {
   return t;
 }
 
-template <int kF16>
+template <int kF16, int kBN>
 __global__ void __launch_bounds__(LG_THREADS, 1) lf_gemm_kernel(const __grid_constant__ LgParams P) {
+  using Lay = LgLayout<kBN>;
   extern __shared__ __align__(1024) uint8_t lg_smem_raw[];
   const uint32_t sbase = lf_smem(lg_smem_raw);
   if (sbase & 1023u) {  // 128-byte swizzled tiles need a 1024-byte aligned window
@@ -132,11 +157,11 @@ __global__ void __launch_bounds__(LG_THREADS, 1) lf_gemm_kernel(const __grid_con
     return;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar = sbase + LG_BAR;
+  const uint32_t bar = sbase + Lay::BAR;
   const uint32_t full0 = bar, empty0 = bar + 8 * LG_NS, acc_full0 = bar + 16 * LG_NS,
                  acc_empty0 = acc_full0 + 16, end_bar = acc_full0 + 32;
-  uint32_t *tmem_slot = (uint32_t *)(lg_smem_raw + LG_BAR + 512);
-  volatile int *abort_flag = (volatile int *)(lg_smem_raw + LG_BAR + 520);  // [2]: flag, wait limit
+  uint32_t *tmem_slot = (uint32_t *)(lg_smem_raw + Lay::BAR + 512);
+  volatile int *abort_flag = (volatile int *)(lg_smem_raw + Lay::BAR + 520);  // [2]: flag, wait limit
   if (threadIdx.x == 0) {
     for (int s = 0; s < LG_NS; s++) {
       lf_mbar_init(full0 + 8 * s, 1);
@@ -181,13 +206,13 @@ __global__ void __launch_bounds__(LG_THREADS, 1) lf_gemm_kernel(const __grid_con
             ok = false;
             break;
           }
-          const uint32_t sa = sbase + s * LG_STAGE, sb = sa + LG_A_BYTES;
-          lf_mbar_expect_tx(full0 + 8 * s, LG_STAGE);
+          const uint32_t sa = sbase + s * Lay::STAGE, sb = sa + LG_A_BYTES;
+          lf_mbar_expect_tx(full0 + 8 * s, Lay::STAGE);
           if (P.mode == 0)
             lg_tma3(sa, &P.map_a, full0 + 8 * s, ks * LG_BK, t.mb * LG_BM, t.b);
           else
             lf_tma_load4(sa, &P.map_a, full0 + 8 * s, 0, t.mb * LG_BM, ks, t.b);
-          lg_tma2(sb, &P.map_b, full0 + 8 * s, ks * LG_BK, t.nb * LG_BN);
+          lg_tma2(sb, &P.map_b, full0 + 8 * s, ks * LG_BK, t.nb * kBN);
         }
       }
       if (*abort_flag) {
@@ -198,7 +223,7 @@ __global__ void __launch_bounds__(LG_THREADS, 1) lf_gemm_kernel(const __grid_con
     }
   } else if (warp == 1) {
     // ================================================== MMA issuer
-    const uint32_t idesc = lf_idesc(kF16, LG_BN, 0);
+    const uint32_t idesc = lf_idesc(kF16, kBN, 0);
     int g = 0, it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < P.tiles && ok; tile += gridDim.x, it++) {
@@ -217,8 +242,8 @@ __global__ void __launch_bounds__(LG_THREADS, 1) lf_gemm_kernel(const __grid_con
           break;
         }
         lf_tc_fence_after();
-        const uint32_t sa = sbase + s * LG_STAGE;
-        lg_mma_k64(tmem + buf * LG_BN, lf_sdesc(sa, 16, 1024), lf_sdesc(sa + LG_A_BYTES, 16, 1024),
+        const uint32_t sa = sbase + s * Lay::STAGE;
+        lg_mma_k64(tmem + buf * kBN, lf_sdesc(sa, 16, 1024), lf_sdesc(sa + LG_A_BYTES, 16, 1024),
                    idesc, ks > 0 ? 1u : 0u, empty0 + 8 * s);
       }
       if (ok) lf_commit_w(acc_full0 + 8 * buf);
@@ -234,7 +259,8 @@ __global__ void __launch_bounds__(LG_THREADS, 1) lf_gemm_kernel(const __grid_con
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int hw = P.H * LF_HD;  // features per projection (head split)
-    int it = 0;
+    const bool issuer = warp == 2 && lane == 0;  // issues the TMA stores
+    int it = 0, nstore = 0;
     for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, it++) {
       const int buf = it & 1;
       if (!lf_wait_warp(acc_full0 + 8 * buf, (it >> 1) & 1, abort_flag, P.status, 46)) break;
@@ -244,65 +270,95 @@ __global__ void __launch_bounds__(LG_THREADS, 1) lf_gemm_kernel(const __grid_con
       const int nvalid = P.row_count ? P.row_count[t.b] : P.L;
       const bool valid = r < nvalid && r < P.L;
       const int orow = valid ? (P.row_map ? P.row_map[(size_t)t.b * P.L + r] : r) : 0;
-      const uint32_t tacc = tmem + lane_off + buf * LG_BN;
-      uint32_t x[2][32];
-      lf_tmem_ld32_nowait(tacc, x[0]);
+      const uint32_t tacc = tmem + lane_off + buf * kBN;
+      // the tile in four 64-column boxes (one head of one projection each in
+      // the head split), each in two 32-column TMEM loads
+      for (int hb = 0; hb < kBN / 64; hb++) {
+        const int n0 = t.nb * kBN + 64 * hb;
+        uint32_t x[2][32];
+        lf_tmem_ld32_nowait(tacc + 64 * hb, x[0]);
+        lf_tmem_ld32_nowait(tacc + 64 * hb + 32, x[1]);
+        lf_tmem_wait_ld_regs(x[0]);
+        lf_tmem_pin_regs(x[1]);
+        if (hb == kBN / 64 - 1) {
+          // every column of the accumulator is in registers: the MMA warp
+          // may start the tile after next in it
+          lf_tc_fence_before();
+          __syncwarp();
+          if (lane == 0) lf_mbar_arrive(acc_empty0 + 8 * buf);
+        }
+        uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < LG_BN / 32; c++) {
-        uint32_t(&v)[32] = x[c & 1];
-        lf_tmem_wait_ld_regs(v);
-        if (c + 1 < LG_BN / 32) lf_tmem_ld32_nowait(tacc + 32 * (c + 1), x[(c + 1) & 1]);
-        const int n0 = t.nb * LG_BN + 32 * c;
-        float bsum[32];
-        if (P.bias) {
-          const uint4 *bp = reinterpret_cast<const uint4 *>(P.bias + n0);
+        for (int hf = 0; hf < 2; hf++) {
+          float bv[32];
+          if (P.bias) {
+            const uint4 *bp = reinterpret_cast<const uint4 *>(P.bias + n0 + 32 * hf);
 #pragma unroll
-          for (int q = 0; q < 4; q++) {
-            const uint4 u = __ldg(bp + q);
-            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+            for (int q = 0; q < 4; q++) {
+              const uint4 u = __ldg(bp + q);
+              const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int e = 0; e < 4; e++) {
-              float lo, hi;
-              if (kF16) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w4[e]));
-                lo = f.x;
-                hi = f.y;
-              } else {
-                lo = __uint_as_float(w4[e] << 16);
-                hi = __uint_as_float(w4[e] & 0xffff0000u);
+              for (int e = 0; e < 4; e++) {
+                if (kF16) {
+                  const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w4[e]));
+                  bv[8 * q + 2 * e] = f.x;
+                  bv[8 * q + 2 * e + 1] = f.y;
+                } else {
+                  bv[8 * q + 2 * e] = __uint_as_float(w4[e] << 16);
+                  bv[8 * q + 2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
+                }
               }
-              bsum[8 * q + 2 * e] = lo;
-              bsum[8 * q + 2 * e + 1] = hi;
             }
-          }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; k++) bsum[k] = 0.f;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 16; k++)
-          pk[k] = lf_pack2<kF16>(__uint_as_float(v[2 * k]) + bsum[2 * k],
-                                 __uint_as_float(v[2 * k + 1]) + bsum[2 * k + 1]);
-        if (valid && n0 < P.N) {
-          uint16_t *dst;
-          if (P.out_mode == 0) {
-            const int p = n0 / hw, hn = n0 - p * hw, h = hn / LF_HD, c0 = hn - h * LF_HD;
-            dst = reinterpret_cast<uint16_t *>(P.outs[p]) +
-                  (((size_t)t.b * P.H + h) * P.Lout + orow) * LF_HD + c0;
           } else {
-            dst = reinterpret_cast<uint16_t *>(P.outs[0]) + ((size_t)t.b * P.L + orow) * P.N + n0;
-          }
-          uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-          for (int q = 0; q < 4; q++) d4[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            for (int k = 0; k < 32; k++) bv[k] = 0.f;
+          }
+#pragma unroll
+          for (int k = 0; k < 16; k++)
+            pk[16 * hf + k] = lf_pack2<kF16>(__uint_as_float(x[hf][2 * k]) + bv[2 * k],
+                                             __uint_as_float(x[hf][2 * k + 1]) + bv[2 * k + 1]);
         }
+        if (P.row_map) {
+          // selected rows: scattered to their positions, 128 bytes per row
+          if (valid) {
+            const int p = n0 / hw, hn = n0 - p * hw, h = hn / LF_HD;
+            uint4 *d4 = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(P.outs[p]) +
+                                                  (((size_t)t.b * P.H + h) * P.Lout + orow) * LF_HD);
+#pragma unroll
+            for (int q = 0; q < 8; q++) d4[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
+          continue;
+        }
+        // staged in shared memory in the 128-byte swizzle layout, then one
+        // TMA store of the 128 x 64 box (rows past the tensor are clipped)
+        const int sb = nstore & 1;
+        const uint32_t stg = sbase + Lay::STG + sb * (LG_BM * 128);
+        if (issuer && nstore >= 2)
+          asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");  // box nstore-2 read out
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+        for (int q = 0; q < 8; q++) {
+          const uint32_t a = stg + row * 128 + ((q ^ (row & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * q]),
+                       "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
+                       : "memory");
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (issuer) {
+          if (P.out_mode == 0) {
+            const int p = n0 / hw, hn = n0 - p * hw, h = hn / LF_HD;
+            lg_store4(&P.map_out[p], stg, 0, t.mb * LG_BM, h, t.b);
+          } else {
+            lg_store3(&P.map_out[0], stg, n0, t.mb * LG_BM, t.b);
+          }
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+        nstore++;
       }
-      // accumulator read out: the MMA warp may start the tile after next in it
-      lf_tc_fence_before();
-      __syncwarp();
-      if (lane == 0) lf_mbar_arrive(acc_empty0 + 8 * buf);
     }
+    // the stores must be complete (not only read out) before the kernel ends
+    if (issuer) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
 
   // ---------------------------------------------------- teardown
@@ -395,6 +451,13 @@ static bool lg_make_map(CUtensorMap *m, int f16, const void *base, int rank, con
 
 static size_t lg_align(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Output tile width: 256 features, unless that leaves more than a quarter of
+// the SMs without a tile (then 128: twice the tiles).  N is a multiple of 256.
+static int lg_tile_width(int mtiles, int N) {
+  const long long t256 = (long long)mtiles * (N / 256);
+  return t256 * 4 >= 3LL * lf_sm_count() ? 256 : 128;
+}
+
 struct LgWs {
   size_t count, rows, xs, total;
 };
@@ -450,15 +513,17 @@ static int lg_cuda(cudaError_t e, const char *what) {
   return lf_record_error(LF_ERR_CUDA, msg);
 }
 
-static int lg_launch(LgParams &P, int f16, cudaStream_t stream, bool pdl) {
-  void (*kern)(const LgParams) = f16 ? lf_gemm_kernel<1> : lf_gemm_kernel<0>;
+static int lg_launch(LgParams &P, int f16, int bn, cudaStream_t stream, bool pdl) {
+  void (*kern)(const LgParams) = bn == 256 ? (f16 ? lf_gemm_kernel<1, 256> : lf_gemm_kernel<0, 256>)
+                                           : (f16 ? lf_gemm_kernel<1, 128> : lf_gemm_kernel<0, 128>);
+  const int smem = bn == 256 ? LgLayout<256>::SMEM : LgLayout<128>::SMEM;
   int st;
-  if ((st = lg_cuda(lf_kernel_smem((const void *)kern, LG_SMEM), "cudaFuncSetAttribute"))) return st;
+  if ((st = lg_cuda(lf_kernel_smem((const void *)kern, smem), "cudaFuncSetAttribute"))) return st;
   const unsigned grid = (unsigned)std::max(1, std::min(P.tiles, lf_sm_count()));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(LG_THREADS);
-  cfg.dynamicSmemBytes = LG_SMEM;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -541,7 +606,8 @@ extern "C" int lf_proj_in(const lf_proj_params *p, int nproj, const void *x, con
   }
   P.ksteps = K / LG_BK;
   P.mblk = (P.L + LG_BM - 1) / LG_BM;
-  P.nblk = P.N / LG_BN;
+  const int bn = lg_tile_width(P.B * P.mblk, P.N);
+  P.nblk = P.N / bn;
   P.tiles = P.B * P.mblk * P.nblk;
   {
     const cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)P.L, (cuuint64_t)P.B};
@@ -553,11 +619,17 @@ extern "C" int lf_proj_in(const lf_proj_params *p, int nproj, const void *x, con
   {
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)P.N};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {LG_BK, LG_BN};
+    const cuuint32_t box[2] = {LG_BK, (cuuint32_t)bn};
     if (!lg_make_map(&P.map_b, f16, w_in, 2, dims, strides, box))
       return lf_record_error(LF_ERR_CUDA, "projection: tensor map encode failed (w_in)");
   }
-  return lg_launch(P, f16, stream, rows_mask != nullptr);
+  if (!rows_mask) {
+    for (int i = 0; i < nproj; i++)
+      if (!lf_make_map(&P.map_out[i], f16, outs[i], (uint64_t)p->n, (uint64_t)p->H, (uint64_t)p->B,
+                       128, (uint64_t)p->n * 128, (uint64_t)p->H * p->n * 128, LG_BM))
+        return lf_record_error(LF_ERR_CUDA, "projection: tensor map encode failed (outs)");
+  }
+  return lg_launch(P, f16, bn, stream, rows_mask != nullptr);
 }
 
 extern "C" int lf_proj_out(const lf_proj_params *p, const void *o, const void *w_out,
@@ -587,7 +659,8 @@ extern "C" int lf_proj_out(const lf_proj_params *p, const void *o, const void *w
   P.status = (int32_t *)workspace;
   P.ksteps = p->H;  // one head per k-step
   P.mblk = (P.L + LG_BM - 1) / LG_BM;
-  P.nblk = P.N / LG_BN;
+  const int bn = lg_tile_width(P.B * P.mblk, P.N);
+  P.nblk = P.N / bn;
   P.tiles = P.B * P.mblk * P.nblk;
   if (!lf_make_map(&P.map_a, f16, o, (uint64_t)p->n, (uint64_t)p->H, (uint64_t)p->B, 128,
                    (uint64_t)p->n * 128, (uint64_t)p->H * p->n * 128, LG_BM))
@@ -595,9 +668,16 @@ extern "C" int lf_proj_out(const lf_proj_params *p, const void *o, const void *w
   {
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)P.N};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {LG_BK, LG_BN};
+    const cuuint32_t box[2] = {LG_BK, (cuuint32_t)bn};
     if (!lg_make_map(&P.map_b, f16, w_out, 2, dims, strides, box))
       return lf_record_error(LF_ERR_CUDA, "projection: tensor map encode failed (w_out)");
   }
-  return lg_launch(P, f16, stream, false);
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)P.L, (cuuint64_t)P.B};
+    const cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)P.L * K * 2};
+    const cuuint32_t box[3] = {64, LG_BM, 1};
+    if (!lg_make_map(&P.map_out[0], f16, y, 3, dims, strides, box))
+      return lf_record_error(LF_ERR_CUDA, "projection: tensor map encode failed (y)");
+  }
+  return lg_launch(P, f16, bn, stream, false);
 }

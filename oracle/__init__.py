@@ -58,7 +58,8 @@ def _load():
         lib.lf_oracle_fwd_head.argtypes = [i32, i32, i32, i32, i32, dbl, p] + [p] * 6 + [p, p]
         lib.lf_oracle_bwd_head.argtypes = [i32, i32, i32, i32, i32, dbl, p] + [p] * 7 + [p] * 6
         lib.lf_oracle_linear.argtypes = [i32, i32, i32, p, p, p, p]
-        for f in ("pattern", "count_pairs", "probs_row", "fwd_head", "bwd_head", "linear"):
+        lib.lf_oracle_cross_head.argtypes = [i32, i32, i32, dbl, p, p, p, p, p, p]
+        for f in ("pattern", "count_pairs", "probs_row", "fwd_head", "bwd_head", "linear", "cross_head"):
             getattr(lib, "lf_oracle_" + f).restype = i32
         _lib = lib
     return _lib
@@ -199,4 +200,34 @@ def linear(x, w, b=None) -> np.ndarray:
     y = np.zeros((M, N), dtype=np.float64)
     _check(_load().lf_oracle_linear(M, N, K, _ptr(xb), _ptr(w), None if bb is None else _ptr(bb), _ptr(y)))
     return y.reshape(lead + (N,))
+
+
+def cross_head(scale: float, kmask, q, k, v):
+    """Cross-attention of one head: q [Lq, hd] against k, v [Lk, hd], keys
+    with kmask != 0 (kmask None: every key).  Returns (o [Lq, hd], lse [Lq])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    Lq, hd = q.shape
+    Lk = k.shape[0]
+    assert k.shape == (Lk, hd) and v.shape == (Lk, hd)
+    m = None if kmask is None else _mask(kmask)
+    assert m is None or m.shape == (Lk,)
+    o = np.zeros((Lq, hd), dtype=np.float64)
+    lse = np.zeros(Lq, dtype=np.float64)
+    _check(_load().lf_oracle_cross_head(Lq, Lk, hd, float(scale), None if m is None else _ptr(m),
+                                        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse)))
+    return o, lse
+
+
+def cross(scale: float, kmask, q, k, v, heads=None):
+    """Cross-attention over q [B, H, Lq, hd] and k, v [B, H, Lk, hd] with a
+    key mask [B, Lk] (or None); ``heads`` = optional list of (b, h) to
+    evaluate (the others are left as NaN).  Returns (o, lse)."""
+    B, H, Lq, hd = np.shape(q)
+    o = np.full((B, H, Lq, hd), np.nan)
+    lse = np.full((B, H, Lq), np.nan)
+    sel = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    for b, h in sel:
+        o[b, h], lse[b, h] = cross_head(scale, None if kmask is None else kmask[b], q[b, h], k[b, h],
+                                        v[b, h])
+    return o, lse
 

@@ -372,3 +372,48 @@ int lf_oracle_linear(int M, int N, int K, const double *x, const double *w, cons
   }
   return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------
+ * Cross-attention of the LED decoder (segmentfault page, section
+ * Longformer-Encoder-Decoder: the decoder attends the whole encoder output
+ * with full attention).  One head: Lq decoder queries against Lk encoder
+ * keys, every key whose kmask entry is nonzero (kmask may be NULL: all):
+ *
+ *   s_ij = scale * <q_i, k_j>,  o_i = sum_j softmax_j(s_ij) v_j,
+ *   lse_i = log sum_j exp(s_ij)
+ *
+ * A query with no valid key gets o_i = 0 and lse_i = -inf.  Double
+ * precision, queries in parallel.
+ * ------------------------------------------------------------------------ */
+int lf_oracle_cross_head(int Lq, int Lk, int hd, double scale, const int32_t *kmask,
+                         const double *q, const double *k, const double *v, double *o,
+                         double *lse) {
+  if (Lq < 0 || Lk < 0 || hd < 1 || !q || !k || !v || !o || !lse) return ORC_ERR_ARG;
+#pragma omp parallel for schedule(dynamic, 8)
+  for (int i = 0; i < Lq; i++) {
+    const double *qi = q + (size_t)i * hd;
+    double *oi = o + (size_t)i * hd;
+    double mx = -INFINITY;
+    for (int j = 0; j < Lk; j++) {
+      if (kmask && kmask[j] == 0) continue;
+      double s = scale * orc_dot(qi, k + (size_t)j * hd, hd);
+      if (s > mx) mx = s;
+    }
+    for (int c = 0; c < hd; c++) oi[c] = 0.0;
+    if (mx == -INFINITY) { /* no valid key */
+      lse[i] = -INFINITY;
+      continue;
+    }
+    double sum = 0.0;
+    for (int j = 0; j < Lk; j++) {
+      if (kmask && kmask[j] == 0) continue;
+      double p = exp(scale * orc_dot(qi, k + (size_t)j * hd, hd) - mx);
+      sum += p;
+      const double *vj = v + (size_t)j * hd;
+      for (int c = 0; c < hd; c++) oi[c] += p * vj[c];
+    }
+    for (int c = 0; c < hd; c++) oi[c] /= sum;
+    lse[i] = mx + log(sum);
+  }
+  return ORC_OK;
+}

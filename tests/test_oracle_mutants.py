@@ -35,6 +35,9 @@ MUTANTS = {
     "linear_weight_transposed": ("for (int k = 0; k < K; k++) s += xr[k] * wr[k];",
                                  "for (int k = 0; k < K; k++) s += xr[k] * w[(size_t)k * N + c];"),
     "linear_bias_dropped": ("y[(size_t)m * N + c] = s + (b ? b[c] : 0.0);", "y[(size_t)m * N + c] = s;"),
+    "cross_mask_ignored": ("if (kmask && kmask[j] == 0) continue;\n      double s = scale",
+                           "if (0) continue;\n      double s = scale"),
+    "cross_unnormalised": ("for (int c = 0; c < hd; c++) oi[c] /= sum;", ""),
     "bwd_dq_unscaled": ("for (int c = 0; c < hd; c++) dq[c] += scale * ds * kj[c];",
                         "for (int c = 0; c < hd; c++) dq[c] += ds * kj[c];"),
 }
@@ -56,6 +59,7 @@ def _pins():
         (pins.test_backward_finite_differences, ("dilated",)),
         (pins.test_backward_zero_rows, ()),
         (pins.test_linear_matches_numpy_and_special_cases, ()),
+        (pins.test_cross_attention_dense_numpy_and_global_row_equivalence, ()),
     ]
 
 
@@ -72,7 +76,8 @@ def test_mutant_is_caught(name, monkeypatch):
         subprocess.check_call(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", so, c, "-lm"])
         real = oracle._load()
         lib = ctypes.CDLL(so)
-        for f in ("threads", "pattern", "count_pairs", "probs_row", "fwd_head", "bwd_head", "linear"):
+        for f in ("threads", "pattern", "count_pairs", "probs_row", "fwd_head", "bwd_head", "linear",
+                  "cross_head"):
             fn = getattr(lib, "lf_oracle_" + f)
             ref = getattr(real, "lf_oracle_" + f)
             fn.restype = ref.restype

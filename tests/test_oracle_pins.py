@@ -321,3 +321,48 @@ def test_linear_matches_numpy_and_special_cases():
     x2 = rng.standard_normal((3, 5, 6))
     np.testing.assert_allclose(oracle.linear(2.5 * x + x2, w), 2.5 * oracle.linear(x, w) + oracle.linear(x2, w),
                                rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------ cross-attention
+
+def test_cross_attention_dense_numpy_and_global_row_equivalence():
+    """oracle.cross_head (LED decoder cross-attention) against a dense numpy
+    softmax attention over the valid keys, and against the oracle's own
+    self-attention where they coincide: a global query row attends every
+    valid key with the global projections, so its output equals cross-
+    attention of that query over K_g, V_g with the mask as the key mask."""
+    rng = np.random.default_rng(11)
+    Lq, Lk, hd, scale = 7, 40, 16, 0.25
+    q, k, v = (rng.standard_normal((L, hd)) for L in (Lq, Lk, Lk))
+    km = np.ones(Lk, np.int32)
+    km[[3, 17, 39]] = 0
+    o, lse = oracle.cross_head(scale, km, q, k, v)
+    s = scale * q @ k.T
+    s[:, km == 0] = -np.inf
+    mx = s.max(axis=1, keepdims=True)
+    p = np.exp(s - mx)
+    np.testing.assert_allclose(o, (p / p.sum(axis=1, keepdims=True)) @ v, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, mx[:, 0] + np.log(p.sum(axis=1)), rtol=0, atol=1e-12)
+    # no key mask = every key
+    o2, _ = oracle.cross_head(scale, None, q, k, v)
+    s2 = scale * q @ k.T
+    p2 = np.exp(s2 - s2.max(axis=1, keepdims=True))
+    np.testing.assert_allclose(o2, (p2 / p2.sum(axis=1, keepdims=True)) @ v, rtol=0, atol=1e-12)
+    # every key masked: o = 0, lse = -inf
+    o3, lse3 = oracle.cross_head(scale, np.zeros(Lk, np.int32), q, k, v)
+    assert np.all(o3 == 0) and np.all(np.isneginf(lse3))
+    # the global-row special case of the self-attention oracle
+    n = 50
+    mask = np.ones(n, np.int32)
+    mask[[0, 21]] = 2
+    mask[45:] = 0
+    t = {nm: rng.standard_normal((n, hd)) for nm in ("qs", "ks", "vs", "qg", "kg", "vg")}
+    fo, flse = oracle.fwd_head(4, 1, False, scale, mask, t["qs"], t["ks"], t["vs"], t["qg"], t["kg"], t["vg"])
+    co, clse = oracle.cross_head(scale, (mask != 0).astype(np.int32), t["qg"][[0, 21]], t["kg"], t["vg"])
+    np.testing.assert_allclose(co, fo[[0, 21]], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(clse, flse[[0, 21]], rtol=0, atol=1e-12)
+    # permuting the keys with their values leaves every output unchanged
+    perm = rng.permutation(Lk)
+    o4, lse4 = oracle.cross_head(scale, km[perm], q, k[perm], v[perm])
+    np.testing.assert_allclose(o4, o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse4, lse, rtol=0, atol=1e-12)

@@ -133,6 +133,37 @@ int lf_attn_decode(const lf_attn_params *p, const void *q, const void *k_cache,
                    const void *v_cache, const int32_t *lengths, void *o,
                    float *lse, void *stream);
 
+/* Cross-attention of the LED decoder: the decoder's queries attend the
+ * whole encoder output with full (dense) attention ("Longformer：处理长文档的
+ * Transformer模型", segmentfault, section Longformer-Encoder-Decoder; the LED
+ * note of the allenai README copy on gittoolsai: inputs up to 16K tokens).
+ * For every (b, h) and decoder position i < Lq:
+ *   s_ij = scale * <q_i, k_j> over the encoder positions j < Lk with
+ *   key_mask[b, j] != 0 (key_mask NULL: every j),
+ *   o_i = sum_j softmax_j(s_ij) v_j,  lse_i = log sum_j exp(s_ij);
+ * a query with no valid key gets o_i = 0, lse_i = -inf.
+ *   q  [B,H,Lq,64], k, v [B,H,Lk,64]; o [B,H,Lq,64] (overwritten); lse
+ *   float32 [B,H,Lq] or NULL; key_mask int32 [B,Lk] or NULL (device).
+ * bf16 / f16 only (tensor cores); the key range of each 128-query block is
+ * split over the SMs and the partial results merged (split-KV).
+ * workspace: ws_bytes >= lf_attn_cross_workspace_size(p); device-side
+ * problems go to its status word (lf_attn_status). */
+typedef struct lf_cross_params {
+  int B;        /* batch size, >= 1 */
+  int H;        /* heads, 1..128 */
+  int Lq;       /* decoder positions (queries) per sequence, >= 1 */
+  int Lk;       /* encoder positions (keys) per sequence, >= 1 */
+  int head_dim; /* must be 64 */
+  float scale;  /* score scale; 0 => 1/sqrt(head_dim) */
+  int dtype;    /* LF_BF16 or LF_F16 */
+} lf_cross_params;
+
+size_t lf_attn_cross_workspace_size(const lf_cross_params *p);
+
+int lf_attn_cross_fwd(const lf_cross_params *p, const void *q, const void *k, const void *v,
+                      const int32_t *key_mask, void *o, float *lse, void *workspace,
+                      size_t ws_bytes, void *stream);
+
 /* Attended (query, key) pairs per (b, h) -> counts int64 [B, H] (device),
  * enumerated with the tile walk and predicates of the forward kernels.
  * workspace: >= lf_attn_workspace_size(p, 0). */

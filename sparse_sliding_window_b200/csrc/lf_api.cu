@@ -323,6 +323,94 @@ extern "C" int lf_attn_mask_dump(const lf_attn_params *p, const int32_t *mask, u
   return lf_cuda(lf_launch_dump(L, out), "dump");
 }
 
+// ---------------------------------------------------------- cross-attention
+
+// Parameters and workspace of lf_attn_cross_fwd: the forward's global-row
+// work items with n = Lk keys and G = Lq query rows.  The key range of a
+// 128-row query block is split so that there are about four work items per
+// SM of a full B200 (148 SMs; a fixed count keeps the workspace size a
+// function of the params alone): at most every 128-key tile its own chunk.
+static int lf_cross_prepare(const lf_cross_params *p, LfDev &dev, LfWs &ws) {
+  g_err[0] = 0;
+  if (!p) return lf_fail(LF_ERR_INVALID, "params is NULL");
+  if (p->B < 1 || p->H < 1 || p->Lq < 1 || p->Lk < 1)
+    return lf_fail(LF_ERR_INVALID, "B, H, Lq, Lk must be >= 1");
+  if (p->H > LF_MAX_H) return lf_fail(LF_ERR_UNSUPPORTED, "H = %d > %d", p->H, LF_MAX_H);
+  if (p->head_dim != LF_HD) return lf_fail(LF_ERR_UNSUPPORTED, "head_dim must be 64 (got %d)", p->head_dim);
+  if (p->dtype != LF_BF16 && p->dtype != LF_F16)
+    return lf_fail(LF_ERR_INVALID, "cross-attention takes LF_BF16 or LF_F16");
+  if (!(p->scale >= 0.f) || isinf(p->scale)) return lf_fail(LF_ERR_INVALID, "scale must be finite and >= 0");
+  if ((long long)p->B * p->H * std::max(p->Lq, p->Lk) > (1ll << 31) - 64)
+    return lf_fail(LF_ERR_UNSUPPORTED, "B*H*L too large");
+  memset(&dev, 0, sizeof(dev));
+  dev.B = p->B;
+  dev.H = p->H;
+  dev.n = p->Lk;
+  dev.G = p->Lq;
+  dev.Gk = (p->Lq + 15) / 16 * 16;
+  dev.cross = 1;
+  dev.scale = p->scale > 0.f ? p->scale : 1.f / sqrtf((float)p->head_dim);
+  dev.scale_log2 = dev.scale * LF_LOG2E;
+  const long long rowblocks = (long long)p->B * p->H * ((p->Lq + LF_BQ - 1) / LF_BQ);
+  const int ktiles = (p->Lk + LF_BK - 1) / LF_BK;
+  const int want = (int)std::min<long long>(ktiles, std::max<long long>(1, (4 * 148 + rowblocks - 1) / rowblocks));
+  dev.chunk_tiles = (ktiles + want - 1) / want;
+  dev.nch = (ktiles + dev.chunk_tiles - 1) / dev.chunk_tiles;
+  const size_t B = p->B, H = p->H, Lq = p->Lq;
+  size_t off = 0;
+  ws = LfWs{};
+  ws.status = off;
+  ws.status_bytes = LF_ST_WORDS * 4;
+  off = lf_align(off + ws.status_bytes);
+  ws.binfo = off;
+  off = lf_align(off + B * LF_BI_WORDS * 4);
+  ws.gidx = ws.grank = ws.qg_c = ws.ks_c = ws.vs_c = ws.delta = off;
+  ws.part_acc = off;
+  off = lf_align(off + B * H * Lq * dev.nch * LF_HD * 4);
+  ws.part_ml = off;
+  off = lf_align(off + B * H * Lq * dev.nch * 8);
+  ws.total = off;
+  ws.G = p->Lq;
+  ws.Gk = dev.Gk;
+  ws.nch = dev.nch;
+  return LF_OK;
+}
+
+extern "C" size_t lf_attn_cross_workspace_size(const lf_cross_params *p) {
+  LfDev dev;
+  LfWs ws;
+  if (lf_cross_prepare(p, dev, ws) != LF_OK) return 0;
+  return ws.total;
+}
+
+extern "C" int lf_attn_cross_fwd(const lf_cross_params *p, const void *q, const void *k,
+                                 const void *v, const int32_t *key_mask, void *o, float *lse,
+                                 void *workspace, size_t ws_bytes, void *stream) {
+  int st;
+  if ((st = lf_check_ptr(q, "q")) || (st = lf_check_ptr(k, "k")) || (st = lf_check_ptr(v, "v")) ||
+      (st = lf_check_ptr(o, "o")) || (st = lf_check_ptr(lse, "lse", true)) ||
+      (st = lf_check_ptr(key_mask, "key_mask", true)))
+    return st;
+  LfLaunch L;
+  if ((st = lf_cross_prepare(p, L.dev, L.ws))) return st;
+  if (!workspace) return lf_fail(LF_ERR_INVALID, "workspace is NULL");
+  if (((uintptr_t)workspace) & 255) return lf_fail(LF_ERR_INVALID, "workspace is not 256-byte aligned");
+  if (ws_bytes < L.ws.total)
+    return lf_fail(LF_ERR_INVALID, "workspace too small (%zu < %zu)", ws_bytes, L.ws.total);
+  L.ws_base = (char *)workspace;
+  L.stream = (cudaStream_t)stream;
+  L.dtype = p->dtype;
+  L.dev.mask = key_mask;
+  L.dev.status = (int32_t *)(L.ws_base + L.ws.status);
+  L.dev.binfo = (int32_t *)(L.ws_base + L.ws.binfo);
+  L.dev.gidx = L.dev.grank = nullptr;
+  L.dev.wait_us = g_test_wait_us;
+  L.dev.skip_tile = g_test_skip_tile;
+  if ((st = lf_cuda(cudaMemsetAsync(L.dev.status, 0, L.ws.status_bytes, L.stream), "status reset")))
+    return st;
+  return lf_tc_cross_fwd(L, q, k, v, o, lse, g_ev_start, g_ev_stop, g_err, sizeof(g_err));
+}
+
 extern "C" int lf_attn_status(void *workspace, void *stream) {
   g_err[0] = 0;
   if (!workspace) return lf_fail(LF_ERR_INVALID, "workspace is NULL");

@@ -62,6 +62,8 @@ struct LfDev {
   int wait_us;    // device wait limit in microseconds (0: default); a test hook
   int skip_tile;  // > 0: CTA 0 of the forward omits the K/V load of its tile
                   // skip_tile - 1, so a bounded wait expires (a test hook)
+  int cross;      // 1: cross-attention (queries = G rows of their own tensor,
+                  // keys = n rows; output rows are the query rows)
   int dil[LF_MAX_H];
 };
 
@@ -175,6 +177,7 @@ struct LfLaunch {
 };
 
 cudaError_t lf_launch_mask_pass(const LfLaunch &L);
+cudaError_t lf_launch_cross_setup(const LfLaunch &L);
 cudaError_t lf_launch_mask_gather(const LfLaunch &L, const void *qg, const void *ks, const void *vs,
                                   void *qg_c, void *ks_c, void *vs_c, int Ga, int Gka);
 cudaError_t lf_launch_count(const LfLaunch &L, int64_t *counts);

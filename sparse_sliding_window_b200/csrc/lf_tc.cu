@@ -732,6 +732,8 @@ __global__ void __launch_bounds__(256)
   const int ng = D.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
   if (e >= ng) return;
   const size_t base = ((size_t)bh * D.G + e) * D.nch;
+  // the output row: the global token's position, or (cross-attention) the query row
+  const size_t orow = D.cross ? (size_t)bh * D.G + e : (size_t)bh * D.n + D.gidx[(size_t)b * D.G + e];
   float m = -INFINITY;
   for (int c = 0; c < D.nch; c++) m = fmaxf(m, part_ml[base + c].x);
   float L = 0.f, a0 = 0.f, a1 = 0.f;
@@ -744,10 +746,10 @@ __global__ void __launch_bounds__(256)
     a0 += acc.x * f;
     a1 += acc.y * f;
   }
-  const int g = D.gidx[(size_t)b * D.G + e];
-  const size_t orow = (size_t)bh * D.n + g;
-  LfIo<T>::st2(o + orow * LF_HD + 2 * lane, a0 / L, a1 / L);
-  if (lse && lane == 0) lse[orow] = (m + log2f(L)) * LF_LN2;
+  // a row with no valid key (cross-attention with every key masked): 0, -inf
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  LfIo<T>::st2(o + orow * LF_HD + 2 * lane, a0 * inv, a1 * inv);
+  if (lse && lane == 0) lse[orow] = L > 0.f ? (m + log2f(L)) * LF_LN2 : -INFINITY;
 }
 
 // ------------------------------------------------------------ host side
@@ -962,3 +964,113 @@ too_big:
                         "dilations must stay <= %d)", (LF_TC_MAX_MAPS - 5) / 3);
   return LF_ERR_UNSUPPORTED;
 }
+
+// ------------------------------------------------------------ cross-attention
+
+// One block per sequence b: the sequence info the global-row work items read
+// (number of query rows, valid keys = key_mask != 0, or all when no mask).
+__global__ void __launch_bounds__(256) lf_cross_setup_kernel(LfDev D) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int b = blockIdx.x;
+  int c = 0;
+  if (D.mask) {
+    const int32_t *m = D.mask + (size_t)b * D.n;
+    for (int j = threadIdx.x; j < D.n; j += blockDim.x) c += m[j] != 0;
+  } else if (threadIdx.x == 0) {
+    c = D.n;
+  }
+  __shared__ int s_c;
+  if (threadIdx.x == 0) s_c = 0;
+  __syncthreads();
+  atomicAdd(&s_c, c);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t *bi = D.binfo + (size_t)b * LF_BI_WORDS;
+    bi[LF_BI_NG] = D.G;
+    bi[LF_BI_NVALID] = s_c;
+    bi[LF_BI_GMIN] = 0;
+    bi[LF_BI_GMAX] = D.G - 1;
+  }
+}
+
+cudaError_t lf_launch_cross_setup(const LfLaunch &L) {
+  lf_cross_setup_kernel<<<L.dev.B, 256, 0, L.stream>>>(L.dev);
+  lf_launches_add(1);
+  return cudaGetLastError();
+}
+
+int lf_tc_cross_fwd(const LfLaunch &L, const void *q, const void *k, const void *v, void *o,
+                    float *lse, cudaEvent_t ev_start, cudaEvent_t ev_stop, char *err, size_t errlen) {
+  const LfDev &D = L.dev;
+  const int f16 = L.dtype == LF_F16 ? 1 : 0;
+  LfTcParams P;
+  memset(&P, 0, sizeof(P));
+  P.dev = D;
+  P.f16 = f16;
+  const uint64_t H = D.H, B = D.B, rowb = 128;
+  // every work item is a global-row item: 128 query rows x one key chunk
+  P.nseg = 0;
+  P.per_batch = 0;
+  P.map_kg = 0;
+  P.map_vg = 1;
+  P.map_qgc = 2;
+  P.map_ksc = 0;  // (global-column tiles do not occur)
+  P.map_vsc = 1;
+  P.gbox = LF_BK;
+  const uint64_t Lk = D.n, Lq = D.G;
+  if (!lf_make_map(&P.maps[0], f16, k, Lk, H, B, rowb, Lk * rowb, H * Lk * rowb, LF_BK) ||
+      !lf_make_map(&P.maps[1], f16, v, Lk, H, B, rowb, Lk * rowb, H * Lk * rowb, LF_BK) ||
+      !lf_make_map(&P.maps[2], f16, q, Lq, H, B, rowb, Lq * rowb, H * Lq * rowb, LF_BQ)) {
+    snprintf(err, errlen, "cross-attention: tensor map encode failed");
+    return LF_ERR_CUDA;
+  }
+  P.ngq = (D.G + LF_BQ - 1) / LF_BQ;
+  P.n_gitems = D.B * D.H * P.ngq * D.nch;
+  P.o = o;
+  P.lse = lse;
+  P.part_acc = (float *)(L.ws_base + L.ws.part_acc);
+  P.part_ml = (float2 *)(L.ws_base + L.ws.part_ml);
+  cudaError_t e = lf_launch_cross_setup(L);
+  if (e != cudaSuccess) {
+    snprintf(err, errlen, "cross setup launch: %s", cudaGetErrorString(e));
+    return LF_ERR_CUDA;
+  }
+  void (*kern)(const LfTcParams) = f16 ? lf_tc_fwd_kernel<1> : lf_tc_fwd_kernel<0>;
+  if ((e = lf_kernel_smem((const void *)kern, LF_SMEM_BYTES)) != cudaSuccess) {
+    snprintf(err, errlen, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    return LF_ERR_CUDA;
+  }
+  const long long items = P.n_gitems;
+  const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>(items, lf_sm_count()));
+  P.sched_cta = items <= 4LL * grid ? 1 : 0;
+  if (ev_start && ev_stop) cudaEventRecord(ev_start, L.stream);
+  cudaError_t le = lf_launch_pdl((const void *)kern, grid, LF_TC_THREADS, LF_SMEM_BYTES, L.stream, &P);
+  lf_launches_add(1);
+  if (ev_start && ev_stop) cudaEventRecord(ev_stop, L.stream);
+  e = le != cudaSuccess ? le : cudaGetLastError();
+  if (e != cudaSuccess) {
+    snprintf(err, errlen, "cross-attention launch: %s", cudaGetErrorString(e));
+    return LF_ERR_CUDA;
+  }
+  const long long rows = (long long)D.B * D.H * D.G;
+  const unsigned cgrid = (unsigned)((rows + 7) / 8);
+  const float *pacc = (const float *)P.part_acc;
+  const float2 *pml = (const float2 *)P.part_ml;
+  if (f16) {
+    __half *oo = (__half *)o;
+    void *args[] = {(void *)&D, (void *)&pacc, (void *)&pml, (void *)&oo, (void *)&lse};
+    le = lf_launch_pdl_args((const void *)lf_combine_kernel<__half>, cgrid, 256, 0, L.stream, args);
+  } else {
+    __nv_bfloat16 *oo = (__nv_bfloat16 *)o;
+    void *args[] = {(void *)&D, (void *)&pacc, (void *)&pml, (void *)&oo, (void *)&lse};
+    le = lf_launch_pdl_args((const void *)lf_combine_kernel<__nv_bfloat16>, cgrid, 256, 0, L.stream, args);
+  }
+  lf_launches_add(1);
+  e = le != cudaSuccess ? le : cudaGetLastError();
+  if (e != cudaSuccess) {
+    snprintf(err, errlen, "combine launch: %s", cudaGetErrorString(e));
+    return LF_ERR_CUDA;
+  }
+  return LF_OK;
+}
+

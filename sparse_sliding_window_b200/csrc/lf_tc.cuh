@@ -41,6 +41,12 @@ struct LfTcBwdArgs {
 // Enqueue the tensor-core backward (after the mask pass).
 int lf_tc_bwd(const LfLaunch &L, const LfTcBwdArgs &a, char *err, size_t errlen);
 
+// Enqueue the cross-attention forward: the global-row work items of the
+// forward kernel over every query row of q against k / v (L.dev.cross = 1,
+// n = keys, G = queries), then the split-KV merge.
+int lf_tc_cross_fwd(const LfLaunch &L, const void *q, const void *k, const void *v, void *o,
+                    float *lse, cudaEvent_t ev_start, cudaEvent_t ev_stop, char *err, size_t errlen);
+
 // Enqueue the tensor-core forward (after the mask pass).  Returns an LF_*
 // code; on failure writes a message into err.
 int lf_tc_fwd(const LfLaunch &L, const LfTcArgs &a, char *err, size_t errlen);

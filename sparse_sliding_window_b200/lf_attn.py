@@ -25,7 +25,7 @@ EXPORTS = ["lf_attn_version", "lf_attn_workspace_size", "lf_attn_fwd", "lf_attn_
            "lf_attn_count_pairs", "lf_attn_mask_dump", "lf_attn_status",
            "lf_attn_set_timing_events", "lf_attn_launch_count", "lf_attn_last_error",
            "lf_attn_fwd_noalloc", "lf_attn_status_noalloc", "lf_attn_decode",
-           "lf_attn_set_test_hooks"]
+           "lf_attn_set_test_hooks", "lf_attn_cross_workspace_size", "lf_attn_cross_fwd"]
 # every symbol include/lf_proj.h declares
 PROJ_EXPORTS = ["lf_proj_workspace_size", "lf_proj_in", "lf_proj_out", "lf_proj_set_timing_events"]
 LF_STATIC_WORKSPACE_BYTES = 16 << 20
@@ -43,6 +43,11 @@ class lf_attn_params(ctypes.Structure):
                 ("dilation", ctypes.POINTER(ctypes.c_int32)), ("causal", ctypes.c_int),
                 ("scale", ctypes.c_float), ("dtype", ctypes.c_int), ("max_global", ctypes.c_int),
                 ("kernel", ctypes.c_int)]
+
+
+class lf_cross_params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("Lq", ctypes.c_int), ("Lk", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("scale", ctypes.c_float), ("dtype", ctypes.c_int)]
 
 
 class lf_proj_params(ctypes.Structure):
@@ -82,6 +87,11 @@ def load(path: str = LIB_PATH):
         lib.lf_attn_status_noalloc.restype = i32
         for f in ("fwd", "bwd", "count_pairs", "mask_dump", "status", "set_timing_events"):
             getattr(lib, "lf_attn_" + f).restype = i32
+        CP = ctypes.POINTER(lf_cross_params)
+        lib.lf_attn_cross_workspace_size.argtypes = [CP]
+        lib.lf_attn_cross_workspace_size.restype = sz
+        lib.lf_attn_cross_fwd.argtypes = [CP, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.lf_attn_cross_fwd.restype = i32
         PP = ctypes.POINTER(lf_proj_params)
         lib.lf_proj_workspace_size.argtypes = [PP, i32]
         lib.lf_proj_workspace_size.restype = sz
@@ -207,6 +217,32 @@ def lf_attn_set_timing_events(ev_start, ev_stop):
 
 def lf_attn_launch_count() -> int:
     return int(load().lf_attn_launch_count())
+
+
+def make_cross_params(B: int, H: int, Lq: int, Lk: int, dtype: int = LF_BF16, scale: float = 0.0,
+                      head_dim: int = 64):
+    p = lf_cross_params()
+    p.B, p.H, p.Lq, p.Lk, p.head_dim, p.scale, p.dtype = B, H, Lq, Lk, head_dim, float(scale), dtype
+    return p
+
+
+def lf_attn_cross_workspace_size(p) -> int:
+    return int(load().lf_attn_cross_workspace_size(ctypes.byref(p)))
+
+
+def cross_workspace(p, device="cuda"):
+    import torch
+    nbytes = lf_attn_cross_workspace_size(p)
+    if nbytes == 0:
+        _check(LF_ERR_INVALID)
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def lf_attn_cross_fwd(p, q, k, v, key_mask, o, lse, ws, stream=None):
+    """LED decoder cross-attention: q [B,H,Lq,64] against k, v [B,H,Lk,64]
+    (keys with key_mask != 0; key_mask None: all) -> o [B,H,Lq,64], lse."""
+    _check(load().lf_attn_cross_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(key_mask), _ptr(o),
+                                    _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def make_proj_params(B: int, n: int, H: int, dtype: int = LF_BF16, head_dim: int = 64):

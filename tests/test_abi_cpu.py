@@ -129,3 +129,22 @@ def test_projection_abi_exports_and_host_checks(lib):
     assert lib.lf_proj_out(ctypes.byref(q), a, a, None, a, a, 16, None) == L.LF_ERR_INVALID
     assert lib.lf_proj_out(ctypes.byref(L.make_proj_params(1, 128, 6, L.LF_BF16)), a, a, None, a, a,
                            4096, None) == L.LF_ERR_UNSUPPORTED
+
+
+def test_cross_attention_workspace_and_host_checks(lib):
+    p = L.make_cross_params(2, 16, 1024, 16384, L.LF_BF16)
+    w = L.lf_attn_cross_workspace_size(p)
+    assert w > 0 and w % 256 == 0
+    assert w >= 2 * 16 * 1024 * 64 * 4  # at least one fp32 partial per query row
+    for bad in (dict(B=0), dict(H=0), dict(Lq=0), dict(Lk=0), dict(dtype=L.LF_F32), dict(head_dim=32),
+                dict(H=200)):
+        kw = dict(B=1, H=2, Lq=100, Lk=300, dtype=L.LF_BF16)
+        kw.update(bad)
+        hd = kw.pop("head_dim", 64)
+        assert L.lf_attn_cross_workspace_size(L.make_cross_params(head_dim=hd, **kw)) == 0, bad
+    buf = (ctypes.c_char * 8192)()
+    a = (ctypes.addressof(buf) + 255) & ~255
+    q = L.make_cross_params(1, 2, 100, 300, L.LF_BF16)
+    assert lib.lf_attn_cross_fwd(ctypes.byref(q), None, a, a, None, a, None, a, 1 << 20, None) == L.LF_ERR_INVALID
+    assert lib.lf_attn_cross_fwd(ctypes.byref(q), a, a + 4, a, None, a, None, a, 1 << 20, None) == L.LF_ERR_INVALID
+    assert lib.lf_attn_cross_fwd(ctypes.byref(q), a, a, a, None, a, None, a, 16, None) == L.LF_ERR_INVALID

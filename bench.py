@@ -435,6 +435,53 @@ def projection_numbers(wl, steps, warmup, dev):
     return res
 
 
+def cross_numbers(steps, warmup, dev, B=2, H=16, Lq=1024, Lk=16384):
+    """LED decoder cross-attention (the pages' 16K-token encoder output,
+    1024 decoder positions, 16 heads, two sequences): lf_attn_cross_fwd,
+    kernel by the library's CUDA events, step (setup + kernel + merge) by
+    events around the call; inputs rotate over enough sets to exceed L2.
+    4 * 64 FLOP per (query, key) pair."""
+    import torch
+    from sparse_sliding_window_b200 import lf_attn as L
+    g = torch.Generator(device=dev).manual_seed(99)
+    set_bytes = B * H * (Lq + 2 * Lk) * 64 * 2
+    nsets = max(2, int(2 * torch.cuda.get_device_properties(dev).L2_cache_size // set_bytes) + 1)
+    sets = [[torch.randn(B, H, L_, 64, device=dev, generator=g).bfloat16() for L_ in (Lq, Lk, Lk)]
+            for _ in range(nsets)]
+    km = torch.ones(B, Lk, dtype=torch.int32, device=dev)
+    o = torch.empty(B, H, Lq, 64, device=dev, dtype=torch.bfloat16)
+    lse = torch.empty(B, H, Lq, device=dev)
+    p = L.make_cross_params(B, H, Lq, Lk, L.LF_BF16)
+    ws = L.cross_workspace(p, device=dev)
+    for i in range(max(3, warmup)):
+        L.lf_attn_cross_fwd(p, *sets[i % nsets], km, o, lse, ws)
+    torch.cuda.synchronize(dev)
+    a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    c.record()
+    kt, st = [], []
+    for i in range(max(5, min(steps, 30))):
+        L.lf_attn_set_timing_events(a, c)
+        s0.record()
+        L.lf_attn_cross_fwd(p, *sets[i % nsets], km, o, lse, ws)
+        s1.record()
+        L.lf_attn_set_timing_events(None, None)
+        torch.cuda.synchronize(dev)
+        kt.append(a.elapsed_time(c) * 1e-3)
+        st.append(s0.elapsed_time(s1) * 1e-3)
+    L.lf_attn_status(ws)
+    kt.sort()
+    st.sort()
+    flops = 4.0 * 64 * B * H * Lq * Lk
+    pk = _peaks()
+    return {"shape": {"B": B, "H": H, "Lq": Lq, "Lk": Lk}, "kernel_us": kt[len(kt) // 2] * 1e6,
+            "step_us": st[len(st) // 2] * 1e6, "tflops_kernel": flops / kt[len(kt) // 2] * 1e-12,
+            "tflops_step": flops / st[len(st) // 2] * 1e-12,
+            "frac_kernel": flops / kt[len(kt) // 2] * 1e-12 / pk["bf16"], "peak_tflops": pk["bf16"],
+            "peak_source": pk["src"], "l2": "inputs rotate over %d sets" % nsets}
+
+
 def run_decode(args, wl):
     import torch
     dev = torch.device("cuda", 0)
@@ -714,6 +761,7 @@ def main():
     del m
     if world == 1 and args.kernel != "simt":
         line["projections"] = projection_numbers(wl, args.steps, args.warmup, dev)
+        line["cross_attention"] = cross_numbers(args.steps, args.warmup, dev)
     if not args.no_others and args.kernel != "simt":
         # every other workload, driver-observed beside the headline: its
         # forward step / main kernel / roofline, the backward where it has

@@ -139,6 +139,52 @@ template <> struct LfIo<__half> {
   }
 };
 
+// 16-byte slice of a 64-element row: N elements of T as floats.  A row is
+// handled by 64 / N consecutive lanes (a lane group).
+template <typename T> struct LfVec;
+template <> struct LfVec<float> {
+  static constexpr int N = 4;
+  static __device__ __forceinline__ void ld(const float *p, float (&x)[4]) {
+    const float4 v = *reinterpret_cast<const float4 *>(p);
+    x[0] = v.x;
+    x[1] = v.y;
+    x[2] = v.z;
+    x[3] = v.w;
+  }
+  static __device__ __forceinline__ void st(float *p, const float (&x)[4]) {
+    *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+  }
+};
+template <typename H2, typename T> struct LfVec16 {
+  static constexpr int N = 8;
+  static __device__ __forceinline__ void ld(const T *p, float (&x)[8]) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const float2 f = LfIo<T>::ld2(reinterpret_cast<const T *>(&w[k]));
+      x[2 * k] = f.x;
+      x[2 * k + 1] = f.y;
+    }
+  }
+  static __device__ __forceinline__ void st(T *p, const float (&x)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) LfIo<T>::st2(reinterpret_cast<T *>(&w[k]), x[2 * k], x[2 * k + 1]);
+    *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+template <> struct LfVec<__nv_bfloat16> : LfVec16<__nv_bfloat162, __nv_bfloat16> {};
+template <> struct LfVec<__half> : LfVec16<__half2, __half> {};
+
+// sum over an aligned group of G lanes (G a power of two dividing 32)
+template <int G>
+__device__ __forceinline__ float lf_group_sum(float v) {
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
 __device__ __forceinline__ float lf_warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

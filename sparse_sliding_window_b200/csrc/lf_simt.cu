@@ -402,17 +402,27 @@ cudaError_t lf_launch_simt_fwd(const LfLaunch &L, const void *qs, const void *ks
 
 // ========================================================= CUDA-core bwd
 
-// delta[row] = sum_c dO[row, c] * O[row, c]   (float32; 0 for mask-0 rows)
+// delta[row] = sum_c dO[row, c] * O[row, c]   (float32; 0 for mask-0 rows).
+// A lane group of 64 / N lanes per row, 16 bytes of O and of dO per lane.
 template <typename T>
 __global__ void __launch_bounds__(256)
     lf_bwd_delta_kernel(LfDev P, const T *o, const T *dO, float *delta) {
-  const int lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (row >= (long long)P.B * P.H * P.n) return;
-  const size_t off = (size_t)row * LF_HD + 2 * lane;
-  float2 a = LfIo<T>::ld2(o + off), g = LfIo<T>::ld2(dO + off);
-  float s = lf_warp_sum(a.x * g.x + a.y * g.y);
-  if (lane == 0) delta[row] = s;
+  constexpr int N = LfVec<T>::N, TPR = LF_HD / N;
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long row = t / TPR;
+  const int part = (int)(t % TPR);
+  const bool in = row < (long long)P.B * P.H * P.n;
+  float s = 0.f;
+  if (in) {
+    float a[N], g[N];
+    const size_t off = (size_t)row * LF_HD + part * N;
+    LfVec<T>::ld(o + off, a);
+    LfVec<T>::ld(dO + off, g);
+#pragma unroll
+    for (int k = 0; k < N; k++) s += a[k] * g[k];
+  }
+  s = lf_group_sum<TPR>(s);
+  if (in && part == 0) delta[row] = s;
 }
 
 // dQ: one warp per query row, same key enumeration as the forward.
@@ -516,58 +526,64 @@ __global__ void __launch_bounds__(256)
   LfIo<T>::st2(dvs + joff, v0, v1);
 }
 
-// dK_g, dV_g: one warp per key row j, over the global rows (every global
-// row attends every valid key through Q_g / K_g / V_g).
+// dK_g, dV_g: one lane group (64 / N lanes, 16 bytes each) per key row j,
+// over the global rows (every global row attends every valid key through
+// Q_g / K_g / V_g); each global row's scores are group sums.  Rows of mask-0
+// keys are zero.
 template <typename T>
 __global__ void __launch_bounds__(256)
     lf_bwd_dkv_g_kernel(LfDev P, const T *qg, const T *kg, const T *vg, const float *lse,
                         const T *dO, const float *delta, T *dkg, T *dvg) {
-  // one warp per 8 consecutive keys j of one (b, h); the global rows' Q_g /
-  // dO rows are shared by the 8 keys, the 8 keys' loads are issued together
-  const int lane = threadIdx.x & 31;
-  const int n = P.n, nb = (n + 7) / 8;
-  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (w >= (long long)P.B * P.H * nb) return;
-  const int jb = (int)(w % nb) * 8;
-  const int bh = (int)(w / nb), b = bh / P.H;
-  const int32_t *m = P.mask + (size_t)b * n;
-  const size_t base = (size_t)bh * n * LF_HD + 2 * lane;
-  float2 kk[8], vv[8];
-  float k0[8], k1[8], v0[8], v1[8];
-  bool on[8];
+  constexpr int N = LfVec<T>::N, TPR = LF_HD / N;
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long key = t / TPR;  // (b, h, j)
+  const int part = (int)(t % TPR);
+  const int n = P.n;
+  const bool in = key < (long long)P.B * P.H * n;
+  const long long kk = in ? key : 0;
+  const int j = (int)(kk % n);
+  const int bh = (int)(kk / n), b = bh / P.H;
+  const bool on = in && P.mask[(size_t)b * n + j] != 0;
+  float kx[N], vx[N], ak[N], av[N];
 #pragma unroll
-  for (int u = 0; u < 8; u++) {
-    const int j = min(jb + u, n - 1);
-    kk[u] = LfIo<T>::ld2(kg + base + (size_t)j * LF_HD);
-    vv[u] = LfIo<T>::ld2(vg + base + (size_t)j * LF_HD);
-    on[u] = jb + u < n && m[j] != 0;
-    k0[u] = k1[u] = v0[u] = v1[u] = 0.f;
-  }
+  for (int k = 0; k < N; k++) ak[k] = av[k] = 0.f;
+  const size_t joff = (size_t)kk * LF_HD + part * N;
+  LfVec<T>::ld(kg + joff, kx);
+  LfVec<T>::ld(vg + joff, vx);
+  // every lane of the warp runs the same global-row loop (group sums); a
+  // warp's keys may belong to two (b, h): the longer count is walked
   const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
-  const int32_t *gl = P.gidx + (size_t)b * P.G;
-  for (int t = 0; t < ng; t++) {
-    const int i = gl[t];
-    const size_t ioff = base + (size_t)i * LF_HD, ir = (size_t)bh * n + i;
-    const float2 q = LfIo<T>::ld2(qg + ioff), g = LfIo<T>::ld2(dO + ioff);
-    const float L2 = lse[ir] * LF_LOG2E, Dg = delta[ir];
+  int ngw = ng;
 #pragma unroll
-    for (int u = 0; u < 8; u++) {
-      if (!on[u]) continue;
-      const float2 sd = lf_warp_sum2(q.x * kk[u].x + q.y * kk[u].y, g.x * vv[u].x + g.y * vv[u].y);
-      const float pr = exp2f(sd.x * P.scale_log2 - L2);
-      const float ds = pr * (sd.y - Dg) * P.scale;
-      k0[u] += ds * q.x;
-      k1[u] += ds * q.y;
-      v0[u] += pr * g.x;
-      v1[u] += pr * g.y;
+  for (int o = 16; o > 0; o >>= 1) ngw = max(ngw, __shfl_xor_sync(0xffffffffu, ngw, o));
+  const int32_t *gl = P.gidx + (size_t)b * P.G;
+  for (int e = 0; e < ngw; e++) {
+    const bool act = on && e < ng;
+    const int i = act ? gl[e] : 0;
+    float q[N], g[N];
+    const size_t ioff = ((size_t)bh * n + i) * LF_HD + part * N, ir = (size_t)bh * n + i;
+    LfVec<T>::ld(qg + ioff, q);
+    LfVec<T>::ld(dO + ioff, g);
+    float s = 0.f, dp = 0.f;
+#pragma unroll
+    for (int k = 0; k < N; k++) {
+      s += q[k] * kx[k];
+      dp += g[k] * vx[k];
+    }
+    s = lf_group_sum<TPR>(s);
+    dp = lf_group_sum<TPR>(dp);
+    if (!act) continue;
+    const float pr = exp2f(s * P.scale_log2 - lse[ir] * LF_LOG2E);
+    const float ds = pr * (dp - delta[ir]) * P.scale;
+#pragma unroll
+    for (int k = 0; k < N; k++) {
+      ak[k] += ds * q[k];
+      av[k] += pr * g[k];
     }
   }
-#pragma unroll
-  for (int u = 0; u < 8; u++) {
-    if (jb + u >= n) break;
-    const size_t joff = base + (size_t)(jb + u) * LF_HD;
-    LfIo<T>::st2(dkg + joff, k0[u], k1[u]);
-    LfIo<T>::st2(dvg + joff, v0[u], v1[u]);
+  if (in) {
+    LfVec<T>::st(dkg + joff, ak);
+    LfVec<T>::st(dvg + joff, av);
   }
 }
 
@@ -579,15 +595,16 @@ static cudaError_t lf_simt_bwd_t(const LfLaunch &L, const void *qs, const void *
   long long rows = (long long)L.dev.B * L.dev.H * L.dev.n;
   unsigned grid = (unsigned)((rows + 7) / 8);
   float *delta = (float *)(L.ws_base + L.ws.delta);
-  lf_bwd_delta_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)o, (const T *)dO, delta);
+  lf_bwd_delta_kernel<T><<<(unsigned)((rows * (LF_HD / LfVec<T>::N) + 255) / 256), 256, 0, L.stream>>>(
+      L.dev, (const T *)o, (const T *)dO, delta);
   lf_bwd_dq_kernel<T><<<grid, 256, 0, L.stream>>>(
       L.dev, (const T *)qs, (const T *)ks, (const T *)vs, (const T *)qg, (const T *)kg,
       (const T *)vg, lse, (const T *)dO, delta, (T *)dqs, (T *)dqg);
   lf_bwd_dkv_s_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)qs, (const T *)ks,
                                                      (const T *)vs, lse, (const T *)dO, delta,
                                                      (T *)dks, (T *)dvs);
-  const long long w8 = (long long)L.dev.B * L.dev.H * ((L.dev.n + 7) / 8);  // 8 keys per warp
-  lf_bwd_dkv_g_kernel<T><<<(unsigned)((w8 + 7) / 8), 256, 0, L.stream>>>(L.dev, (const T *)qg, (const T *)kg,
+  const unsigned ggrid = (unsigned)((rows * (LF_HD / LfVec<T>::N) + 255) / 256);  // a lane group per key
+  lf_bwd_dkv_g_kernel<T><<<ggrid, 256, 0, L.stream>>>(L.dev, (const T *)qg, (const T *)kg,
                                                      (const T *)vg, lse, (const T *)dO, delta,
                                                      (T *)dkg, (T *)dvg);
   lf_launches_add(4);
@@ -618,10 +635,9 @@ static cudaError_t lf_bwd_delta_dkvg_t(const LfLaunch &L, const void *o, const v
                                        float *delta, const void *qg, const void *kg,
                                        const void *vg, const float *lse, void *dkg, void *dvg) {
   long long rows = (long long)L.dev.B * L.dev.H * L.dev.n;
-  unsigned grid = (unsigned)((rows + 7) / 8);
-  lf_bwd_delta_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)o, (const T *)dO, delta);
-  const long long w8 = (long long)L.dev.B * L.dev.H * ((L.dev.n + 7) / 8);
-  lf_bwd_dkv_g_kernel<T><<<(unsigned)((w8 + 7) / 8), 256, 0, L.stream>>>(L.dev, (const T *)qg, (const T *)kg,
+  const unsigned ggrid = (unsigned)((rows * (LF_HD / LfVec<T>::N) + 255) / 256);  // a lane group per row
+  lf_bwd_delta_kernel<T><<<ggrid, 256, 0, L.stream>>>(L.dev, (const T *)o, (const T *)dO, delta);
+  lf_bwd_dkv_g_kernel<T><<<ggrid, 256, 0, L.stream>>>(L.dev, (const T *)qg, (const T *)kg,
                                                      (const T *)vg, lse, (const T *)dO, delta,
                                                      (T *)dkg, (T *)dvg);
   lf_launches_add(2);

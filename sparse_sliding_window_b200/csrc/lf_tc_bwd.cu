@@ -458,158 +458,261 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
 
 // Global-column part of dK_s / dV_s: a global key g is attended by every
 // local row, by its window or by its global column (union); the band kernel
-// covered the window, this pass the rows whose window misses g.  One warp per
-// (b, h, global e, chunk of rows); partial sums, reduced by lf_bwd_gcol_reduce.
+// covered the window, this pass the rows whose window misses g.  One block of
+// 256 threads per (b, h, global e, chunk of LF_BW_ROWS_PER_CHUNK rows),
+// grid-strided: a lane group (64 / N lanes, 16 bytes of a row each) per row,
+// the groups' sums added in a fixed order into the chunk's partial, which
+// lf_bwd_gcol_reduce adds up.
 template <typename T>
 __global__ void __launch_bounds__(256)
     lf_bwd_gcol_kernel(LfDev P, const T *qs, const T *ks, const T *vs, const float *lse,
                        const T *dO, const float *delta, float *part, int nch) {
-  const int lane = threadIdx.x & 31;
-  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (w >= (long long)P.B * P.H * P.G * nch) return;
-  const int c = (int)(w % nch);
-  const long long be = w / nch;
-  const int e = (int)(be % P.G);
-  const long long bh = be / P.G;
-  const int h = (int)(bh % P.H), b = (int)(bh / P.H), d = P.dil[h], n = P.n;
-  const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
-  float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
-  if (e < ng) {
-    const int g = P.gidx[(size_t)b * P.G + e];
-    const int32_t *m = P.mask + (size_t)b * n;
-    const size_t base = (size_t)bh * n * LF_HD + 2 * lane;
-    const float2 kk = LfIo<T>::ld2(ks + base + (size_t)g * LF_HD);
-    const float2 vv = LfIo<T>::ld2(vs + base + (size_t)g * LF_HD);
-    const int i0 = c * LF_BW_ROWS_PER_CHUNK, i1 = min(n, i0 + LF_BW_ROWS_PER_CHUNK);
-    // rows in batches of 8: every load of a batch is issued before the first
-    // use (a row outside the chunk reads row i1 - 1 and is skipped); the sums
-    // run in row order as before
-    for (int ib = i0; ib < i1; ib += 8) {
-      float2 q[8], go[8];
-      float ls[8], dl[8];
+  constexpr int N = LfVec<T>::N, TPR = LF_HD / N, GPB = 256 / TPR;
+  __shared__ float s_red[8][2 * LF_HD];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = threadIdx.x / TPR, pi = threadIdx.x % TPR;
+  const long long units = (long long)P.B * P.H * P.G * nch;
+  for (long long un = blockIdx.x; un < units; un += gridDim.x) {
+    const int c = (int)(un % nch);
+    const long long be = un / nch;
+    const int e = (int)(be % P.G);
+    const long long bh = be / P.G;
+    const int h = (int)(bh % P.H), b = (int)(bh / P.H), d = P.dil[h], n = P.n;
+    const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
+    float ak[N], av[N];
 #pragma unroll
-      for (int u = 0; u < 8; u++) {
-        const int i = min(ib + u, i1 - 1);
-        const size_t ioff = base + (size_t)i * LF_HD, ir = (size_t)bh * n + i;
-        q[u] = LfIo<T>::ld2(qs + ioff);
-        go[u] = LfIo<T>::ld2(dO + ioff);
-        ls[u] = lse[ir];
-        dl[u] = delta[ir];
-      }
+    for (int k = 0; k < N; k++) ak[k] = av[k] = 0.f;
+    if (e < ng) {
+      const int g = P.gidx[(size_t)b * P.G + e];
+      const int32_t *m = P.mask + (size_t)b * n;
+      const size_t base = (size_t)bh * n * LF_HD + pi * N;
+      float kx[N], vx[N];
+      LfVec<T>::ld(ks + base + (size_t)g * LF_HD, kx);
+      LfVec<T>::ld(vs + base + (size_t)g * LF_HD, vx);
+      const int i0 = c * LF_BW_ROWS_PER_CHUNK, i1 = min(n, i0 + LF_BW_ROWS_PER_CHUNK);
+      for (int rr = 0; rr < LF_BW_ROWS_PER_CHUNK; rr += GPB) {
+        const int i = i0 + rr + grp;
+        const bool valid = i < i1;
+        const int ic = valid ? i : i1 - 1;
+        float q[N], go[N];
+        LfVec<T>::ld(qs + base + (size_t)ic * LF_HD, q);
+        LfVec<T>::ld(dO + base + (size_t)ic * LF_HD, go);
+        float s = 0.f, dp = 0.f;
 #pragma unroll
-      for (int u = 0; u < 8; u++) {
-        const int i = ib + u;
-        if (i >= i1 || m[i] != 1 || lf_in_window(i, g, P.r, d, P.causal)) continue;
-        const float2 sd = lf_warp_sum2(q[u].x * kk.x + q[u].y * kk.y, go[u].x * vv.x + go[u].y * vv.y);
-        const float pr = exp2f(sd.x * P.scale_log2 - ls[u] * LF_LOG2E);
-        const float ds = pr * (sd.y - dl[u]) * P.scale;
-        k0 += ds * q[u].x;
-        k1 += ds * q[u].y;
-        v0 += pr * go[u].x;
-        v1 += pr * go[u].y;
+        for (int k = 0; k < N; k++) {
+          s += q[k] * kx[k];
+          dp += go[k] * vx[k];
+        }
+        s = lf_group_sum<TPR>(s);
+        dp = lf_group_sum<TPR>(dp);
+        if (!valid || m[i] != 1 || lf_in_window(i, g, P.r, d, P.causal)) continue;
+        const size_t ir = (size_t)bh * n + i;
+        const float pr = exp2f(s * P.scale_log2 - lse[ir] * LF_LOG2E);
+        const float ds = pr * (dp - delta[ir]) * P.scale;
+#pragma unroll
+        for (int k = 0; k < N; k++) {
+          ak[k] += ds * q[k];
+          av[k] += pr * go[k];
+        }
       }
     }
+    // the groups of a warp, then the warps in order
+#pragma unroll
+    for (int o = TPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int k = 0; k < N; k++) {
+        ak[k] += __shfl_xor_sync(0xffffffffu, ak[k], o);
+        av[k] += __shfl_xor_sync(0xffffffffu, av[k], o);
+      }
+    if (lane < TPR)
+#pragma unroll
+      for (int k = 0; k < N; k++) {
+        s_red[warp][pi * N + k] = ak[k];
+        s_red[warp][LF_HD + pi * N + k] = av[k];
+      }
+    __syncthreads();
+    if (warp == 0) {
+      float *dst = part + (size_t)un * 2 * LF_HD;
+      for (int x = lane; x < 2 * LF_HD; x += 32) {
+        float t = 0.f;
+        for (int w = 0; w < 8; w++) t += s_red[w][x];
+        dst[x] = t;
+      }
+    }
+    __syncthreads();
   }
-  float *dst = part + ((size_t)be * nch + c) * 2 * LF_HD + 2 * lane;
-  *reinterpret_cast<float2 *>(dst) = make_float2(k0, k1);
-  *reinterpret_cast<float2 *>(dst + LF_HD) = make_float2(v0, v1);
 }
 
-// dK_s[g] += sum of chunks; dV_s[g] likewise (one warp per (b, h, e)).
+// dK_s[g] += sum of chunks; dV_s[g] likewise.  One block of LF_BW_RED_WARPS
+// warps per (b, h, e): warp w sums chunks w, w + LF_BW_RED_WARPS, ... in
+// order (four loads in flight), then the warps' sums are added in warp
+// order -- a fixed order, so the result is deterministic.
+#define LF_BW_RED_WARPS 16
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(32 * LF_BW_RED_WARPS)
     lf_bwd_gcol_reduce(LfDev P, const float *part, int nch, T *dks, T *dvs) {
-  const int lane = threadIdx.x & 31;
-  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (w >= (long long)P.B * P.H * P.G) return;
+  __shared__ float4 s_acc[LF_BW_RED_WARPS][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // rows (b, h, e) grid-strided; rows past the sequence's global count skip
+  for (long long w = blockIdx.x; w < (long long)P.B * P.H * P.G; w += gridDim.x) {
   const int e = (int)(w % P.G);
   const long long bh = w / P.G;
   const int b = (int)(bh / P.H);
-  if (e >= P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG]) return;
-  float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
-  for (int c = 0; c < nch; c++) {
-    const float *src = part + ((size_t)w * nch + c) * 2 * LF_HD + 2 * lane;
-    const float2 a = *reinterpret_cast<const float2 *>(src);
-    const float2 v = *reinterpret_cast<const float2 *>(src + LF_HD);
-    k0 += a.x;
-    k1 += a.y;
-    v0 += v.x;
-    v1 += v.y;
+  if (e >= P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG]) continue;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c0 = warp; c0 < nch; c0 += 4 * LF_BW_RED_WARPS) {
+    float2 a[4], v[4];
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+      const int c = min(c0 + u * LF_BW_RED_WARPS, nch - 1);
+      const float *src = part + ((size_t)w * nch + c) * 2 * LF_HD + 2 * lane;
+      a[u] = *reinterpret_cast<const float2 *>(src);
+      v[u] = *reinterpret_cast<const float2 *>(src + LF_HD);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+      if (c0 + u * LF_BW_RED_WARPS >= nch) break;
+      acc.x += a[u].x;
+      acc.y += a[u].y;
+      acc.z += v[u].x;
+      acc.w += v[u].y;
+    }
   }
-  const int g = P.gidx[(size_t)b * P.G + e];
-  const size_t off = ((size_t)bh * P.n + g) * LF_HD + 2 * lane;
-  const float2 kb = LfIo<T>::ld2(dks + off), vb = LfIo<T>::ld2(dvs + off);
-  LfIo<T>::st2(dks + off, kb.x + k0, kb.y + k1);
-  LfIo<T>::st2(dvs + off, vb.x + v0, vb.y + v1);
+  s_acc[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float4 t = s_acc[0][lane];
+    for (int k = 1; k < LF_BW_RED_WARPS; k++) {
+      const float4 x = s_acc[k][lane];
+      t.x += x.x;
+      t.y += x.y;
+      t.z += x.z;
+      t.w += x.w;
+    }
+    const int g = P.gidx[(size_t)b * P.G + e];
+    const size_t off = ((size_t)bh * P.n + g) * LF_HD + 2 * lane;
+    const float2 kb = LfIo<T>::ld2(dks + off), vb = LfIo<T>::ld2(dvs + off);
+    LfIo<T>::st2(dks + off, kb.x + t.x, kb.y + t.y);
+    LfIo<T>::st2(dvs + off, vb.x + t.z, vb.y + t.w);
+  }
+  __syncthreads();  // s_acc is reused by the block's next row
+  }
 }
 
-// dQ_g of the global rows: every valid key through Q_g / K_g / V_g.  One warp
-// per (b, h, global e, chunk of keys); partial sums reduced below.
+// dQ_g of the global rows: every valid key through Q_g / K_g / V_g.  One
+// block per (b, h, global e, chunk of keys), grid-strided, a lane group per
+// key as in lf_bwd_gcol_kernel; partial sums reduced below.
 template <typename T>
 __global__ void __launch_bounds__(256)
     lf_bwd_grow_kernel(LfDev P, const T *qg, const T *kg, const T *vg, const float *lse,
                        const T *dO, const float *delta, float *part, int nch) {
-  const int lane = threadIdx.x & 31;
-  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (w >= (long long)P.B * P.H * P.G * nch) return;
-  const int c = (int)(w % nch);
-  const long long be = w / nch;
-  const int e = (int)(be % P.G);
-  const long long bh = be / P.G;
-  const int b = (int)(bh / P.H), n = P.n;
-  const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
-  float a0 = 0.f, a1 = 0.f;
-  if (e < ng) {
-    const int g = P.gidx[(size_t)b * P.G + e];
-    const int32_t *m = P.mask + (size_t)b * n;
-    const size_t base = (size_t)bh * n * LF_HD + 2 * lane;
-    const size_t gr = (size_t)bh * n + g;
-    const float2 q = LfIo<T>::ld2(qg + base + (size_t)g * LF_HD);
-    const float2 go = LfIo<T>::ld2(dO + base + (size_t)g * LF_HD);
-    const float L2 = lse[gr] * LF_LOG2E, Dg = delta[gr];
-    const int j0 = c * LF_BW_ROWS_PER_CHUNK, j1 = min(n, j0 + LF_BW_ROWS_PER_CHUNK);
-    // keys in batches of 8, every load issued before the first use; sums in key order
-    for (int jb = j0; jb < j1; jb += 8) {
-      float2 k[8], v[8];
+  constexpr int N = LfVec<T>::N, TPR = LF_HD / N, GPB = 256 / TPR;
+  __shared__ float s_red[8][LF_HD];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = threadIdx.x / TPR, pi = threadIdx.x % TPR;
+  const long long units = (long long)P.B * P.H * P.G * nch;
+  for (long long un = blockIdx.x; un < units; un += gridDim.x) {
+    const int c = (int)(un % nch);
+    const long long be = un / nch;
+    const int e = (int)(be % P.G);
+    const long long bh = be / P.G;
+    const int b = (int)(bh / P.H), n = P.n;
+    const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
+    float aq[N];
 #pragma unroll
-      for (int u = 0; u < 8; u++) {
-        const size_t joff = base + (size_t)min(jb + u, j1 - 1) * LF_HD;
-        k[u] = LfIo<T>::ld2(kg + joff);
-        v[u] = LfIo<T>::ld2(vg + joff);
-      }
+    for (int k = 0; k < N; k++) aq[k] = 0.f;
+    if (e < ng) {
+      const int g = P.gidx[(size_t)b * P.G + e];
+      const int32_t *m = P.mask + (size_t)b * n;
+      const size_t base = (size_t)bh * n * LF_HD + pi * N;
+      const size_t gr = (size_t)bh * n + g;
+      float q[N], go[N];
+      LfVec<T>::ld(qg + base + (size_t)g * LF_HD, q);
+      LfVec<T>::ld(dO + base + (size_t)g * LF_HD, go);
+      const float L2 = lse[gr] * LF_LOG2E, Dg = delta[gr];
+      const int j0 = c * LF_BW_ROWS_PER_CHUNK, j1 = min(n, j0 + LF_BW_ROWS_PER_CHUNK);
+      for (int rr = 0; rr < LF_BW_ROWS_PER_CHUNK; rr += GPB) {
+        const int j = j0 + rr + grp;
+        const bool valid = j < j1;
+        const int jc = valid ? j : j1 - 1;
+        float kx[N], vx[N];
+        LfVec<T>::ld(kg + base + (size_t)jc * LF_HD, kx);
+        LfVec<T>::ld(vg + base + (size_t)jc * LF_HD, vx);
+        float s = 0.f, dp = 0.f;
 #pragma unroll
-      for (int u = 0; u < 8; u++) {
-        const int j = jb + u;
-        if (j >= j1 || m[j] == 0) continue;
-        const float2 sd = lf_warp_sum2(q.x * k[u].x + q.y * k[u].y, go.x * v[u].x + go.y * v[u].y);
-        const float pr = exp2f(sd.x * P.scale_log2 - L2);
-        const float ds = pr * (sd.y - Dg) * P.scale;
-        a0 += ds * k[u].x;
-        a1 += ds * k[u].y;
+        for (int k = 0; k < N; k++) {
+          s += q[k] * kx[k];
+          dp += go[k] * vx[k];
+        }
+        s = lf_group_sum<TPR>(s);
+        dp = lf_group_sum<TPR>(dp);
+        if (!valid || m[j] == 0) continue;
+        const float pr = exp2f(s * P.scale_log2 - L2);
+        const float ds = pr * (dp - Dg) * P.scale;
+#pragma unroll
+        for (int k = 0; k < N; k++) aq[k] += ds * kx[k];
       }
     }
+#pragma unroll
+    for (int o = TPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int k = 0; k < N; k++) aq[k] += __shfl_xor_sync(0xffffffffu, aq[k], o);
+    if (lane < TPR)
+#pragma unroll
+      for (int k = 0; k < N; k++) s_red[warp][pi * N + k] = aq[k];
+    __syncthreads();
+    if (warp == 0) {
+      float *dst = part + (size_t)un * LF_HD;
+      for (int x = lane; x < LF_HD; x += 32) {
+        float t = 0.f;
+        for (int w = 0; w < 8; w++) t += s_red[w][x];
+        dst[x] = t;
+      }
+    }
+    __syncthreads();
   }
-  *reinterpret_cast<float2 *>(part + ((size_t)be * nch + c) * LF_HD + 2 * lane) = make_float2(a0, a1);
 }
 
+// dQ_g[g] = sum of chunks: one block per (b, h, e), the order of
+// lf_bwd_gcol_reduce.
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(32 * LF_BW_RED_WARPS)
     lf_bwd_grow_reduce(LfDev P, const float *part, int nch, T *dqg) {
-  const int lane = threadIdx.x & 31;
-  const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (w >= (long long)P.B * P.H * P.G) return;
+  __shared__ float2 s_acc[LF_BW_RED_WARPS][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (long long w = blockIdx.x; w < (long long)P.B * P.H * P.G; w += gridDim.x) {
   const int e = (int)(w % P.G);
   const long long bh = w / P.G;
   const int b = (int)(bh / P.H);
-  if (e >= P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG]) return;
-  float a0 = 0.f, a1 = 0.f;
-  for (int c = 0; c < nch; c++) {
-    const float2 a = *reinterpret_cast<const float2 *>(part + ((size_t)w * nch + c) * LF_HD + 2 * lane);
-    a0 += a.x;
-    a1 += a.y;
+  if (e >= P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG]) continue;
+  float2 acc = make_float2(0.f, 0.f);
+  for (int c0 = warp; c0 < nch; c0 += 4 * LF_BW_RED_WARPS) {
+    float2 a[4];
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+      const int c = min(c0 + u * LF_BW_RED_WARPS, nch - 1);
+      a[u] = *reinterpret_cast<const float2 *>(part + ((size_t)w * nch + c) * LF_HD + 2 * lane);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+      if (c0 + u * LF_BW_RED_WARPS >= nch) break;
+      acc.x += a[u].x;
+      acc.y += a[u].y;
+    }
   }
-  const int g = P.gidx[(size_t)b * P.G + e];
-  LfIo<T>::st2(dqg + ((size_t)bh * P.n + g) * LF_HD + 2 * lane, a0, a1);
+  s_acc[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float2 t = s_acc[0][lane];
+    for (int k = 1; k < LF_BW_RED_WARPS; k++) {
+      t.x += s_acc[k][lane].x;
+      t.y += s_acc[k][lane].y;
+    }
+    const int g = P.gidx[(size_t)b * P.G + e];
+    LfIo<T>::st2(dqg + ((size_t)bh * P.n + g) * LF_HD + 2 * lane, t.x, t.y);
+  }
+  __syncthreads();
+  }
 }
 
 // ============================================== host
@@ -624,13 +727,15 @@ static cudaError_t lf_bwd_global_parts(const LfLaunch &L, const LfTcBwdArgs &a, 
   if (e != cudaSuccess) return e;
   if (D.G > 0) {
     const long long wk = (long long)D.B * D.H * D.G * nch, wr = (long long)D.B * D.H * D.G;
-    lf_bwd_gcol_kernel<T><<<(unsigned)((wk + 7) / 8), 256, 0, L.stream>>>(
+    const unsigned ugrid = (unsigned)std::min<long long>(wk, 148LL * 16);  // grid-strided units
+    lf_bwd_gcol_kernel<T><<<ugrid, 256, 0, L.stream>>>(
         D, (const T *)a.qs, (const T *)a.ks, (const T *)a.vs, a.lse, (const T *)a.dO, delta, part_kv, nch);
-    lf_bwd_gcol_reduce<T><<<(unsigned)((wr + 7) / 8), 256, 0, L.stream>>>(D, part_kv, nch, (T *)a.dks,
-                                                                           (T *)a.dvs);
-    lf_bwd_grow_kernel<T><<<(unsigned)((wk + 7) / 8), 256, 0, L.stream>>>(
+    const unsigned rgrid = (unsigned)std::min<long long>(wr, 4096);
+    lf_bwd_gcol_reduce<T><<<rgrid, 32 * LF_BW_RED_WARPS, 0, L.stream>>>(D, part_kv, nch, (T *)a.dks,
+                                                                        (T *)a.dvs);
+    lf_bwd_grow_kernel<T><<<ugrid, 256, 0, L.stream>>>(
         D, (const T *)a.qg, (const T *)a.kg, (const T *)a.vg, a.lse, (const T *)a.dO, delta, part_q, nch);
-    lf_bwd_grow_reduce<T><<<(unsigned)((wr + 7) / 8), 256, 0, L.stream>>>(D, part_q, nch, (T *)a.dqg);
+    lf_bwd_grow_reduce<T><<<rgrid, 32 * LF_BW_RED_WARPS, 0, L.stream>>>(D, part_q, nch, (T *)a.dqg);
     lf_launches_add(4);
   }
   return cudaGetLastError();

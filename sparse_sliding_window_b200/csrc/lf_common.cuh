@@ -106,6 +106,23 @@ __host__ __device__ __forceinline__ void lf_band_cols(int q, int u, int r, int c
   if (hi > LF_BK - 1) hi = LF_BK - 1;
 }
 
+// The same for column tiles of kW columns (band tile u starts kW*u after
+// the block's first window key): band tiles of a block, and the columns of
+// tile u that row q attends, q <= kW*u + c <= q + (causal ? r : 2r).
+template <int kW>
+__host__ __device__ __forceinline__ int lf_band_tiles_w(int r, int causal) {
+  return (LF_BQ + (causal ? r : 2 * r) + kW - 1) / kW;
+}
+template <int kW>
+__host__ __device__ __forceinline__ void lf_band_cols_w(int q, int u, int r, int causal, int &lo,
+                                                        int &hi) {
+  const int base = kW * u;
+  lo = q - base;
+  if (lo < 0) lo = 0;
+  hi = q + (causal ? r : 2 * r) - base;
+  if (hi > kW - 1) hi = kW - 1;
+}
+
 // Length of residue sub-sequence rho of a length-n sequence with dilation d.
 __host__ __device__ __forceinline__ int lf_sub_len(int n, int d, int rho) {
   return rho < n ? (n - rho + d - 1) / d : 0;

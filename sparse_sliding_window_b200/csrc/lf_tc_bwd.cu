@@ -23,11 +23,18 @@
 //             accumulates dV += P^T dO, dK += dS^T Q.  Writes the band part of
 //             dK_s, dV_s (the global-column part of the global keys is added
 //             afterwards by lf_bwd_gcol_*).
-// Roles per CTA (192 threads, one CTA per SM: all 512 TMEM columns): warps
+// Column tiles are 64 wide (keys in mode Q, queries in mode KV).  Roles per
+// CTA (192 threads, 256 TMEM columns, ~98 KB of shared memory: two CTAs per
+// SM, so one CTA's MMA round trip overlaps the other's exponentials): warps
 // 0-3 form P / dS (one TMEM lane = one row), warp 4 issues TMA loads (row
-// operands once, column operands into a 3-stage ring), warp 5 issues the
-// MMAs.  TMEM: S [0,128), dP [128,256), acc0 [256,320) (dQ or dV),
-// acc1 [320,384) (dK), A0 [384,448) (dS or P^T), A1 [448,512) (dS^T).
+// operands once, column operands into a 4-stage ring), warp 5 issues the
+// MMAs.  TMEM: S [0,64), dP [64,128), acc0 [128,192) (dQ or dV), acc1
+// [192,256) (dK).  The 16-bit A operands of the accumulating products are
+// written over the columns they were computed from, chunk by chunk once
+// read: dS (mode Q) or P^T (mode KV) into S's first 32 columns, dS^T into
+// dP's.  The next tile's S and dP are issued after those products by the
+// same thread, and tcgen05 operations of one thread run in order, so they
+// overwrite the A operands only after they have been read.
 // Every mbarrier wait is bounded (status LF_ERR_DEVICE_TIMEOUT on expiry).
 #include <stdio.h>
 #include <string.h>
@@ -40,28 +47,31 @@
 #include "lf_tc.cuh"
 
 #define LF_BW_THREADS 192
-#define LF_BW_NS 3
+#define LF_BW_NS 4
+#define LF_BW_BK 64  // columns (keys / queries) per column tile
 #define LF_BW_MAX_MAPS 192  // kernel parameters may take up to 32 KB
 #define LF_BW_MAX_SEG 96
 #define LF_BW_ROWS_PER_CHUNK 64  // rows (keys) per warp of the global-row / -column parts
 
 #define LF_BW_R0 0
 #define LF_BW_R1 16384
-#define LF_BW_C0(s) (32768 + (s)*32768)
-#define LF_BW_C1(s) (32768 + (s)*32768 + 16384)
-#define LF_BW_VEC(s) (32768 + LF_BW_NS * 32768 + (s)*1024)
-#define LF_BW_BAR (32768 + LF_BW_NS * 32768 + LF_BW_NS * 1024)
+#define LF_BW_CST (LF_BW_BK * 128 * 2)  // one column stage: two 64-row tiles
+#define LF_BW_C0(s) (32768 + (s)*LF_BW_CST)
+#define LF_BW_C1(s) (32768 + (s)*LF_BW_CST + LF_BW_BK * 128)
+#define LF_BW_VEC(s) (32768 + LF_BW_NS * LF_BW_CST + (s)*(2 * LF_BW_BK * 4))
+#define LF_BW_BAR (32768 + LF_BW_NS * LF_BW_CST + LF_BW_NS * 2 * LF_BW_BK * 4)
 #define LF_BW_SMEM (LF_BW_BAR + 256)
+static_assert(2 * (LF_BW_SMEM + 1024) <= 233472, "two CTAs per SM");
 
 #define LF_BT_S 0
-#define LF_BT_DP 128
-#define LF_BT_ACC0 256
-#define LF_BT_ACC1 320
-#define LF_BT_A0 384
-#define LF_BT_A1 448
+#define LF_BT_DP 64
+#define LF_BT_ACC0 128
+#define LF_BT_ACC1 192
+#define LF_BT_COLS 256
 
 struct LfBwParams {
-  CUtensorMap maps[LF_BW_MAX_MAPS];  // per residue view: q, k, v, dO; then ks_c, vs_c
+  CUtensorMap maps[LF_BW_MAX_MAPS];  // per residue view: q, k, v, dO (128-row boxes), the same
+                                     // with 64-row boxes; then ks_c, vs_c
   LfDev dev;
   LfTcSeg seg[LF_BW_MAX_SEG];
   int nseg, per_batch, gbox, map_ksc, map_vsc;
@@ -91,7 +101,7 @@ __device__ __forceinline__ void lf_bw_decode(const LfBwParams &P, int idx, int m
   it.rho = sg.rho;
   it.cnt = sg.cnt;
   it.map = sg.map;
-  it.nband = lf_band_tiles(D.r, D.causal);
+  it.nband = lf_band_tiles_w<LF_BW_BK>(D.r, D.causal);
   const int32_t *bi = D.binfo + (size_t)it.b * LF_BI_WORDS;
   it.ng = bi[LF_BI_NG];
   it.nglob = 0;
@@ -101,19 +111,19 @@ __device__ __forceinline__ void lf_bw_decode(const LfBwParams &P, int idx, int m
       const int tlast = min(it.row0 + LF_BQ - 1, it.cnt - 1);
       if (bi[LF_BI_GMIN] >= tlast - D.r && bi[LF_BI_GMAX] <= it.row0 + D.r) need = false;
     }
-    it.nglob = need ? (it.ng + LF_BK - 1) / LF_BK : 0;
+    it.nglob = need ? (it.ng + LF_BW_BK - 1) / LF_BW_BK : 0;
   }
   it.T = it.nband + it.nglob;
 }
 
 // first column-operand row of band tile u
 __device__ __forceinline__ int lf_bw_tile_row(const LfDev &D, const LfBwItem &it, int modeq, int u) {
-  if (modeq || !D.causal) return it.row0 - D.r + LF_BK * u;
-  return it.row0 + LF_BK * u;  // causal, rows = keys: queries t in [j, j + r]
+  if (modeq || !D.causal) return it.row0 - D.r + LF_BW_BK * u;
+  return it.row0 + LF_BW_BK * u;  // causal, rows = keys: queries t in [j, j + r]
 }
 
 template <int kF16, int kModeQ>
-__global__ void __launch_bounds__(LF_BW_THREADS, 1)
+__global__ void __launch_bounds__(LF_BW_THREADS, 2)
     lf_tc_bwd_kernel(const __grid_constant__ LfBwParams P) {
   extern __shared__ __align__(1024) uint8_t lf_bw_smem[];
   const uint32_t sbase = lf_smem(lf_bw_smem);
@@ -130,8 +140,8 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
   const int T = it.T;
 
   const uint32_t bar = sbase + LF_BW_BAR;
-  const uint32_t row_full = bar, s_full = bar + 8, ds_full = bar + 16, acc_done = bar + 24,
-                 o_full = bar + 32, end_bar = bar + 40;
+  const uint32_t row_full = bar, s_full = bar + 8, ds_full = bar + 16, o_full = bar + 32,
+                 end_bar = bar + 40;
   const uint32_t col_full0 = bar + 48, col_empty0 = bar + 48 + 8 * LF_BW_NS;
   uint32_t *tmem_slot = (uint32_t *)(gbase + LF_BW_BAR + 192);
   volatile int *abort_flag = (volatile int *)(gbase + LF_BW_BAR + 196);  // [2]: flag, wait limit
@@ -140,7 +150,6 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
     lf_mbar_init(row_full, 1);
     lf_mbar_init(s_full, 1);
     lf_mbar_init(ds_full, 4);
-    lf_mbar_init(acc_done, 1);
     lf_mbar_init(o_full, 1);
     lf_mbar_init(end_bar, 1);
     for (int s = 0; s < LF_BW_NS; s++) {
@@ -155,7 +164,7 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
   if (warp == 5) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      lf_smem(tmem_slot)),
-                 "r"(512)
+                 "r"(LF_BT_COLS)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -170,6 +179,9 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
     // ================================================== TMA producer (+ column vectors)
     const CUtensorMap *mq = &P.maps[it.map], *mk = &P.maps[it.map + 1], *mv = &P.maps[it.map + 2],
                       *mdo = &P.maps[it.map + 3];
+    // the same views with 64-row boxes, for the column tiles
+    const CUtensorMap *cq = &P.maps[it.map + 4], *ck = &P.maps[it.map + 5], *cv = &P.maps[it.map + 6],
+                      *cdo = &P.maps[it.map + 7];
     if (lane == 0) {
       lf_mbar_expect_tx(row_full, 32768);
       lf_tma_load4(sbase + LF_BW_R0, kModeQ ? mq : mk, row_full, 0, it.row0, it.h, it.b);
@@ -186,11 +198,11 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
       uint32_t bytes;
       if (t < it.nband) {
         row = lf_bw_tile_row(D, it, kModeQ, t);
-        c0 = kModeQ ? mk : mq;
-        c1 = kModeQ ? mv : mdo;
-        bytes = 32768;
+        c0 = kModeQ ? ck : cq;
+        c1 = kModeQ ? cv : cdo;
+        bytes = 2 * LF_BW_BK * 128;
       } else {
-        row = (t - it.nband) * LF_BK;
+        row = (t - it.nband) * LF_BW_BK;
         c0 = &P.maps[P.map_ksc];
         c1 = &P.maps[P.map_vsc];
         bytes = 2 * P.gbox * 128;
@@ -199,9 +211,9 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
         // per-column (query) log-normaliser in log2 units and D; +inf marks
         // columns that are not local queries (probability 0)
         float *lse2 = (float *)(gbase + LF_BW_VEC(s));
-        float *dv = lse2 + LF_BQ;
+        float *dv = lse2 + LF_BW_BK;
 #pragma unroll
-        for (int k = 0; k < 4; k++) {
+        for (int k = 0; k < LF_BW_BK / 32; k++) {
           const int c = lane + 32 * k, tq = row + c;
           float l2 = INFINITY, dd = 0.f;
           if (tq >= 0 && tq < it.cnt) {
@@ -239,10 +251,12 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
     const uint64_t dc1mn = lf_sdesc(sbase + LF_BW_C1(0), 0, 1024);
     const uint32_t id_acc = lf_idesc(kF16, 64, 1);
     const int ngk = (it.ng + 15) / 16 * 16;
-    auto ncols = [&](int t) { return t < it.nband ? LF_BK : min(LF_BK, ngk - (t - it.nband) * LF_BK); };
+    auto ncols = [&](int t) {
+      return t < it.nband ? LF_BW_BK : min(LF_BW_BK, ngk - (t - it.nband) * LF_BW_BK);
+    };
     // S = R0 C0^T and dP = R1 C1^T of column tile t -> s_full
     auto issue_s = [&](int t) {
-      const uint64_t so = (uint64_t)((t % LF_BW_NS) * (32768 >> 4));
+      const uint64_t so = (uint64_t)((t % LF_BW_NS) * (LF_BW_CST >> 4));
       lf_mma_s2_phase(tmem + LF_BT_S, dr0, dc0 + so, tmem + LF_BT_DP, dr1, dc1 + so,
                       lf_idesc(kF16, ncols(t), 0), s_full);
     };
@@ -254,27 +268,29 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
       for (int t = 0; t < T; t++) {
         if (!lf_wait_warp(ds_full, t & 1, abort_flag, D.status, 25)) break;
         lf_tc_fence_after();
+        const uint64_t so = (uint64_t)((t % LF_BW_NS) * (LF_BW_CST >> 4));
+        const uint32_t kmask = (1u << (ncols(t) / 16)) - 1u;
+        const uint32_t acc0 = t > 0 ? 1u : 0u;
+        const uint32_t last = t + 1 == T ? o_full : 0u;
+        if (kModeQ) {
+          // dQ += dS K   (dS packed in S's columns; K tile as the MN-major B operand)
+          lf_mma_ts_phase(tmem + LF_BT_ACC0, tmem + LF_BT_S, dc0mn + so, 2048 >> 4, id_acc, kmask,
+                          acc0, col_empty0 + 8 * (t % LF_BW_NS), last, 0u);
+        } else {
+          // dV += P^T dO ; dK += dS^T Q   (P^T in S's columns, dS^T in dP's)
+          lf_mma_ts_phase(tmem + LF_BT_ACC0, tmem + LF_BT_S, dc1mn + so, 2048 >> 4, id_acc, kmask,
+                          acc0, 0u, 0u, 0u);
+          lf_mma_ts_phase(tmem + LF_BT_ACC1, tmem + LF_BT_DP, dc0mn + so, 2048 >> 4, id_acc, kmask,
+                          acc0, col_empty0 + 8 * (t % LF_BW_NS), last, 0u);
+        }
+        // the next tile's S and dP, issued after the products that read this
+        // tile's A operands out of the same columns
         if (t + 1 < T) {
           const int s2 = (t + 1) % LF_BW_NS;
           if (!lf_wait_warp(col_full0 + 8 * s2, ((t + 1) / LF_BW_NS) & 1, abort_flag, D.status, 26))
             break;
           lf_tc_fence_after();
           issue_s(t + 1);
-        }
-        const uint64_t so = (uint64_t)((t % LF_BW_NS) * (32768 >> 4));
-        const uint32_t kmask = (1u << (ncols(t) / 16)) - 1u;
-        const uint32_t acc0 = t > 0 ? 1u : 0u;
-        const uint32_t last = t + 1 == T ? o_full : 0u;
-        if (kModeQ) {
-          // dQ += dS K   (K tile as the MN-major B operand)
-          lf_mma_ts_phase(tmem + LF_BT_ACC0, tmem + LF_BT_A0, dc0mn + so, 2048 >> 4, id_acc, kmask,
-                          acc0, col_empty0 + 8 * (t % LF_BW_NS), acc_done, last);
-        } else {
-          // dV += P^T dO ; dK += dS^T Q
-          lf_mma_ts_phase(tmem + LF_BT_ACC0, tmem + LF_BT_A0, dc1mn + so, 2048 >> 4, id_acc, kmask,
-                          acc0, 0u, 0u, 0u);
-          lf_mma_ts_phase(tmem + LF_BT_ACC1, tmem + LF_BT_A1, dc0mn + so, 2048 >> 4, id_acc, kmask,
-                          acc0, col_empty0 + 8 * (t % LF_BW_NS), acc_done, last);
         }
       }
     }
@@ -286,7 +302,6 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
     const int q = warp * 32 + lane;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const uint32_t tS = tmem + lane_off + LF_BT_S, tDP = tmem + lane_off + LF_BT_DP;
-    const uint32_t tA0 = tmem + lane_off + LF_BT_A0, tA1 = tmem + lane_off + LF_BT_A1;
     const float sl2 = D.scale_log2, scale = D.scale;
     const int trow = it.row0 + q;
     int pos = 0, code = 0;
@@ -316,30 +331,31 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
         break;
       }
       lf_tc_fence_after();
-      uint32_t w[4];
+      constexpr int NC = LF_BW_BK / 32;  // 32-column chunks per tile
+      uint32_t w[NC];
       const int s = t % LF_BW_NS;
       if (t < it.nband) {
         const int kb = lf_bw_tile_row(D, it, kModeQ, t);
         int lo, hi;
-        lf_band_cols(q, t, D.r, D.causal, lo, hi);
+        lf_band_cols_w<LF_BW_BK>(q, t, D.r, D.causal, lo, hi);
         lo = max(lo, -kb);  // column operand rows exist on [0, cnt)
         hi = min(hi, it.cnt - 1 - kb);
         if (!active) hi = -1;
 #pragma unroll
-        for (int cc = 0; cc < 4; cc++) w[cc] = lf_range_bits(lo, hi, 32 * cc);
+        for (int cc = 0; cc < NC; cc++) w[cc] = lf_range_bits(lo, hi, 32 * cc);
         if (kModeQ && padded) {
 #pragma unroll
-          for (int cc = 0; cc < 4; cc++) {
+          for (int cc = 0; cc < NC; cc++) {
             const int tk = kb + 32 * cc + lane;
             const bool okk = tk >= 0 && tk < it.cnt && mrow[it.rho + tk * it.d] != 0;
             w[cc] &= __ballot_sync(0xffffffffu, okk);
           }
         }
       } else {
-        const int gbs = (t - it.nband) * LF_BK;
-        const int hi = active ? min(LF_BK - 1, it.ng - 1 - gbs) : -1;
+        const int gbs = (t - it.nband) * LF_BW_BK;
+        const int hi = active ? min(LF_BW_BK - 1, it.ng - 1 - gbs) : -1;
 #pragma unroll
-        for (int cc = 0; cc < 4; cc++) {
+        for (int cc = 0; cc < NC; cc++) {
           uint32_t inwin = lf_range_bits(e_lo - gbs, e_hi - 1 - gbs, 32 * cc);
           if (it.d > 1) {
             const int e = gbs + 32 * cc + lane;
@@ -358,10 +374,9 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
         }
       }
       const float *clse2 = (const float *)(gbase + LF_BW_VEC(s));
-      const float *cdd = clse2 + LF_BQ;
-      bool gated = (t == 0);
+      const float *cdd = clse2 + LF_BW_BK;
 #pragma unroll
-      for (int cc = 0; cc < 4; cc++) {
+      for (int cc = 0; cc < NC; cc++) {
         uint32_t ds_w[16], p_w[16];
         if (__any_sync(0xffffffffu, w[cc] != 0u)) {
           float x[32], y[32];
@@ -390,19 +405,13 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
 #pragma unroll
           for (int k = 0; k < 16; k++) ds_w[k] = p_w[k] = 0u;
         }
-        if (!gated) {
-          // the previous tile's accumulate MMAs have finished reading A0 / A1
-          if (!lf_wait_warp(acc_done, (t - 1) & 1, abort_flag, D.status, 29)) {
-            alive = false;
-            break;
-          }
-          gated = true;
-        }
+        // packed over columns [16cc, 16cc + 16) of S (and dP): chunk cc's
+        // scores are in registers and chunk cc+1's columns lie beyond them
         if (kModeQ) {
-          lf_tmem_st16(tA0 + 16 * cc, ds_w);
+          lf_tmem_st16(tS + 16 * cc, ds_w);
         } else {
-          lf_tmem_st16(tA0 + 16 * cc, p_w);
-          lf_tmem_st16(tA1 + 16 * cc, ds_w);
+          lf_tmem_st16(tS + 16 * cc, p_w);
+          lf_tmem_st16(tDP + 16 * cc, ds_w);
         }
       }
       if (!alive) break;
@@ -449,7 +458,8 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 1)
   __syncthreads();
   if (warp == 5) {
     lf_tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(LF_BT_COLS)
                  : "memory");
   }
 }
@@ -772,22 +782,22 @@ int lf_tc_bwd(const LfLaunch &L, const LfTcBwdArgs &a, char *err, size_t errlen)
       if (nqb == 0) continue;
       auto key = std::make_pair(d, rho);
       if (!rmap.count(key)) {
-        if (nmaps + 4 > LF_BW_MAX_MAPS - 2) {
+        if (nmaps + 8 > LF_BW_MAX_MAPS - 2) {
           snprintf(err, errlen,
                    "tensor-core backward: too many distinct dilation residues (the sum of the "
-                   "distinct dilations must stay <= %d)", (LF_BW_MAX_MAPS - 2) / 4);
+                   "distinct dilations must stay <= %d)", (LF_BW_MAX_MAPS - 2) / 8);
           return LF_ERR_UNSUPPORTED;
         }
         const char *srcs[4] = {(const char *)a.qs, (const char *)a.ks, (const char *)a.vs,
                                (const char *)a.dO};
-        for (int k = 0; k < 4; k++)
-          if (!lf_make_map(&P.maps[nmaps + k], f16, srcs[k] + rho * rowb, cnt, H, B, d * rowb,
-                           n * rowb, H * n * rowb, LF_BQ)) {
+        for (int k = 0; k < 8; k++)
+          if (!lf_make_map(&P.maps[nmaps + k], f16, srcs[k & 3] + rho * rowb, cnt, H, B, d * rowb,
+                           n * rowb, H * n * rowb, k < 4 ? LF_BQ : LF_BW_BK)) {
             snprintf(err, errlen, "tensor map encode failed (backward, d=%d, rho=%d)", d, rho);
             return LF_ERR_CUDA;
           }
         rmap[key] = nmaps;
-        nmaps += 4;
+        nmaps += 8;
       }
       if (nseg >= LF_BW_MAX_SEG) {
         snprintf(err, errlen, "tensor-core backward: too many head/residue segments");
@@ -803,7 +813,7 @@ int lf_tc_bwd(const LfLaunch &L, const LfTcBwdArgs &a, char *err, size_t errlen)
   P.per_batch = start;
   const int Ga = L.ws.G, Gka = L.ws.Gk;
   char *qg_c = L.ws_base + L.ws.qg_c, *ks_c = L.ws_base + L.ws.ks_c, *vs_c = L.ws_base + L.ws.vs_c;
-  P.gbox = std::min(Gka, LF_BK);
+  P.gbox = std::min(Gka, LF_BW_BK);
   P.map_ksc = nmaps;
   P.map_vsc = nmaps + 1;
   if (!lf_make_map(&P.maps[nmaps], f16, ks_c, Gka, H, B, rowb, Gka * rowb, H * Gka * rowb, P.gbox) ||

@@ -77,8 +77,7 @@ struct LfBwParams {
   int nseg, per_batch, gbox, map_ksc, map_vsc;
   const float *lse;
   const float *delta;
-  void *out0;  // dQ_s (mode Q) or dV_s (mode KV)
-  void *out1;  // dK_s (mode KV)
+  void *dq_out, *dk_out, *dv_out;  // dQ_s (mode Q); dK_s, dV_s (mode KV)
 };
 
 // Work item (shared decode for every role).
@@ -122,10 +121,9 @@ __device__ __forceinline__ int lf_bw_tile_row(const LfDev &D, const LfBwItem &it
   return it.row0 + LF_BW_BK * u;  // causal, rows = keys: queries t in [j, j + r]
 }
 
+// One work item (a 128-row block) of mode kModeQ.
 template <int kF16, int kModeQ>
-__global__ void __launch_bounds__(LF_BW_THREADS, 2)
-    lf_tc_bwd_kernel(const __grid_constant__ LfBwParams P) {
-  extern __shared__ __align__(1024) uint8_t lf_bw_smem[];
+__device__ __forceinline__ void lf_tc_bwd_item(const LfBwParams &P, int item, uint8_t *lf_bw_smem) {
   const uint32_t sbase = lf_smem(lf_bw_smem);
   if (sbase & 1023u) {
     if (threadIdx.x == 0) lf_set_status(P.dev.status, LF_ERR_UNSUPPORTED, 9001);
@@ -136,7 +134,7 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 2)
   const LfDev &D = P.dev;
   const int n = D.n;
   LfBwItem it;
-  lf_bw_decode(P, blockIdx.x, kModeQ, it);
+  lf_bw_decode(P, item, kModeQ, it);
   const int T = it.T;
 
   const uint32_t bar = sbase + LF_BW_BAR;
@@ -433,7 +431,7 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 2)
         lf_tmem_ld32(tmem + lane_off + (which ? LF_BT_ACC1 : LF_BT_ACC0), a);
         lf_tmem_ld32(tmem + lane_off + (which ? LF_BT_ACC1 : LF_BT_ACC0) + 32, c2);
         if (!store) continue;
-        void *outp = which ? P.out1 : P.out0;
+        void *outp = kModeQ ? P.dq_out : (which ? P.dk_out : P.dv_out);
         uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(outp) + orow * LF_HD);
 #pragma unroll
         for (int k = 0; k < 4; k++) {
@@ -462,6 +460,21 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 2)
                  "r"(LF_BT_COLS)
                  : "memory");
   }
+}
+
+// Both modes in one launch: blocks [0, items) are mode KV (dK_s, dV_s),
+// blocks [items, 2 items) mode Q (dQ_s).  The two are independent (both
+// read the forward's lse and the row deltas), so their CTAs share the SMs
+// and fill each other's tails.
+template <int kF16>
+__global__ void __launch_bounds__(LF_BW_THREADS, 2)
+    lf_tc_bwd_kernel(const __grid_constant__ LfBwParams P) {
+  extern __shared__ __align__(1024) uint8_t lf_bw_smem[];
+  const int items = P.dev.B * P.per_batch;
+  if ((int)blockIdx.x < items)
+    lf_tc_bwd_item<kF16, 0>(P, blockIdx.x, lf_bw_smem);
+  else
+    lf_tc_bwd_item<kF16, 1>(P, blockIdx.x - items, lf_bw_smem);
 }
 
 // ============================================== global-token parts (CUDA cores)
@@ -830,18 +843,18 @@ int lf_tc_bwd(const LfLaunch &L, const LfTcBwdArgs &a, char *err, size_t errlen)
       return LF_ERR_CUDA;
     }
   }
-  const unsigned grid = (unsigned)((long long)D.B * P.per_batch);
-  for (int mode = 0; mode < 2; mode++) {  // 0: dK/dV (rows = keys), 1: dQ (rows = queries)
-    void (*kern)(const LfBwParams) =
-        f16 ? (mode ? lf_tc_bwd_kernel<1, 1> : lf_tc_bwd_kernel<1, 0>)
-            : (mode ? lf_tc_bwd_kernel<0, 1> : lf_tc_bwd_kernel<0, 0>);
+  // one launch: dK/dV blocks (rows = keys), then dQ blocks (rows = queries)
+  const unsigned grid = (unsigned)(2LL * D.B * P.per_batch);
+  {
+    void (*kern)(const LfBwParams) = f16 ? lf_tc_bwd_kernel<1> : lf_tc_bwd_kernel<0>;
     ce = lf_kernel_smem((const void *)kern, LF_BW_SMEM);
     if (ce != cudaSuccess) {
       snprintf(err, errlen, "cudaFuncSetAttribute (backward): %s", cudaGetErrorString(ce));
       return LF_ERR_CUDA;
     }
-    P.out0 = mode ? a.dqs : a.dvs;
-    P.out1 = mode ? nullptr : a.dks;
+    P.dq_out = a.dqs;
+    P.dk_out = a.dks;
+    P.dv_out = a.dvs;
     kern<<<grid, LF_BW_THREADS, LF_BW_SMEM, L.stream>>>(P);
     lf_launches_add(1);
     ce = cudaGetLastError();

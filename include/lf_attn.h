@@ -92,8 +92,11 @@ int lf_attn_version(void);
 /* Bytes of device workspace lf_attn_fwd (for_bwd = 0) or lf_attn_bwd
  * (for_bwd = 1) needs for these params; 0 on invalid params.  The caller
  * allocates it (256-byte aligned) and passes it to the call; the library
- * allocates nothing itself.  One workspace must not be used by two calls
- * that may run at the same time. */
+ * allocates nothing itself.  Its first 32 bytes are the device status
+ * word: zero them once after allocating (e.g. cudaMemset); lf_attn_status
+ * zeroes them again after each read, and no call needs them cleared before
+ * it runs.  One workspace must not be used by two calls that may run at the
+ * same time. */
 size_t lf_attn_workspace_size(const lf_attn_params *p, int for_bwd);
 
 /* Forward.  Inputs q_s..v_g [B,H,n,64], mask int32 [B,n] (device).
@@ -178,8 +181,9 @@ int lf_attn_mask_dump(const lf_attn_params *p, const int32_t *mask,
                       void *stream);
 
 /* Synchronise `stream`, read and clear the device status word of
- * `workspace`; returns LF_OK or the first device-side error code
- * (LF_ERR_DEVICE_TIMEOUT, LF_ERR_DEVICE_INPUT, LF_ERR_UNSUPPORTED). */
+ * `workspace`; returns LF_OK or the first device-side error code recorded
+ * since the previous read (LF_ERR_DEVICE_TIMEOUT, LF_ERR_DEVICE_INPUT,
+ * LF_ERR_UNSUPPORTED). */
 int lf_attn_status(void *workspace, void *stream);
 
 /* Optional timing hook: when both are non-NULL cudaEvent_t handles, every
@@ -229,9 +233,9 @@ int lf_attn_fwd_noalloc(const lf_attn_params *p, const void *q_s,
                         void *o, float *lse, void *stream);
 
 /* Synchronise `stream`, read and clear the device status word of the
- * static scratch of lf_attn_fwd_noalloc on the current device.  Every
- * lf_attn_fwd_noalloc clears that word when it starts, so this returns
- * LF_OK or the first device-side error of the latest call on the device
+ * static scratch of lf_attn_fwd_noalloc on the current device (zero when
+ * the library is loaded).  Returns LF_OK or the first device-side error of
+ * the lf_attn_fwd_noalloc calls on the device since the previous read
  * (codes as for lf_attn_status).  Allocates nothing. */
 int lf_attn_status_noalloc(void *stream);
 

@@ -31,7 +31,8 @@
  * Errors: host-side checks return LF_ERR_INVALID (null pointer, bad sizes or
  * alignment, dtype) or LF_ERR_UNSUPPORTED (head_dim != 64, H not a multiple
  * of 4); device-side problems (more selected rows than max_rows, an expired
- * bounded wait) go to the status word of the workspace, read with
+ * bounded wait) go to the status word of the workspace (its first 32 bytes:
+ * zero them once after allocating), read and cleared with
  * lf_attn_status(workspace, stream).  Every call is asynchronous on
  * `stream`; the library allocates nothing.
  */

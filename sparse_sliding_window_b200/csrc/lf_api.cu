@@ -223,9 +223,10 @@ static int lf_bind_ws(const lf_attn_params *p, int for_bwd, void *workspace, siz
   L.dev.grank = (int32_t *)(L.ws_base + L.ws.grank);
   L.dev.wait_us = g_test_wait_us;
   L.dev.skip_tile = g_test_skip_tile;
-  // each call starts with a clear status word (and split counters);
-  // lf_attn_status reads the word back
-  return lf_cuda(cudaMemsetAsync(L.dev.status, 0, L.ws.status_bytes, L.stream), "status reset");
+  // No per-call reset (a memset node before every call): the first kernel
+  // of each call zeroes the work-item counter, and the error word stays set
+  // until lf_attn_status reads and clears it (a fresh workspace starts zeroed)
+  return LF_OK;
 }
 
 extern "C" int lf_attn_fwd(const lf_attn_params *p, const void *q_s, const void *k_s,
@@ -406,8 +407,6 @@ extern "C" int lf_attn_cross_fwd(const lf_cross_params *p, const void *q, const 
   L.dev.gidx = L.dev.grank = nullptr;
   L.dev.wait_us = g_test_wait_us;
   L.dev.skip_tile = g_test_skip_tile;
-  if ((st = lf_cuda(cudaMemsetAsync(L.dev.status, 0, L.ws.status_bytes, L.stream), "status reset")))
-    return st;
   return lf_tc_cross_fwd(L, q, k, v, o, lse, g_ev_start, g_ev_stop, g_err, sizeof(g_err));
 }
 

@@ -548,7 +548,8 @@ static int lg_bind(const lf_proj_params *p, int max_rows, void *workspace, size_
     return lf_record_error(LF_ERR_INVALID, "workspace is not 256-byte aligned");
   w = lg_ws(p, max_rows);
   if (ws_bytes < w.total) return lf_record_error(LF_ERR_INVALID, "workspace too small");
-  return lg_cuda(cudaMemsetAsync(workspace, 0, LF_ST_WORDS * 4, stream), "status reset");
+  (void)stream;
+  return LF_OK;  // the status word stays set until lf_attn_status reads and clears it
 }
 
 extern "C" int lf_proj_in(const lf_proj_params *p, int nproj, const void *x, const void *w_in,

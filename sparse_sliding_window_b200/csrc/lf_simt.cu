@@ -84,6 +84,9 @@ __global__ void __launch_bounds__(1024) lf_mask_pass_kernel(LfDev P) {
   __shared__ typename LfScan::TempStorage tmp;
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = blockIdx.x;
+  // the first kernel of a call: the work-item counter of the forward starts
+  // at zero (read by the kernels after this one completes)
+  if (b == 0 && threadIdx.x == 0) P.status[LF_ST_SCHED] = 0;
   lf_mask_scan(P, b, true, P.gidx + (size_t)b * P.G, tmp);
 }
 
@@ -106,6 +109,7 @@ __global__ void __launch_bounds__(1024)
   extern __shared__ int32_t s_gl[];
   // the forward kernel launched after this one may start its set-up now
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (blockIdx.x == 0 && threadIdx.x == 0) P.status[LF_ST_SCHED] = 0;  // (as lf_mask_pass_kernel)
   const int bh = blockIdx.x, b = bh / P.H;
   const bool tables = bh % P.H == 0;
   const int ng = min(lf_mask_scan(P, b, tables, s_gl, tmp), P.G);

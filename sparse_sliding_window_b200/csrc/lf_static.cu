@@ -78,9 +78,10 @@ extern "C" int lf_attn_fwd_noalloc(const lf_attn_params *p, const void *q_s, con
   void *base = nullptr;
   const int st = lf_static_base(&base, "lf_attn_fwd_noalloc");
   if (st != LF_OK) return st;
-  // The regular forward clears the status word at its start and fully
-  // writes every other scratch region before reading it, so the contents a
-  // previous call left behind never matter.
+  // The regular forward zeroes the work-item counter in its first kernel and
+  // fully writes every other scratch region before reading it; the status
+  // word (zero at load, like every __device__ array) keeps the first error
+  // until lf_attn_status_noalloc reads and clears it.
   return lf_attn_fwd(p, q_s, k_s, v_s, q_g, k_g, v_g, mask, o, lse, base,
                      (size_t)LF_STATIC_WORKSPACE_BYTES, stream);
 }

@@ -972,6 +972,7 @@ too_big:
 __global__ void __launch_bounds__(256) lf_cross_setup_kernel(LfDev D) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = blockIdx.x;
+  if (b == 0 && threadIdx.x == 0) D.status[LF_ST_SCHED] = 0;  // the forward's work-item counter
   int c = 0;
   if (D.mask) {
     const int32_t *m = D.mask + (size_t)b * D.n;

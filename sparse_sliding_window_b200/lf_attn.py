@@ -152,7 +152,7 @@ def workspace(p, for_bwd: bool = False, device="cuda"):
     nbytes = lf_attn_workspace_size(p, for_bwd)
     if nbytes == 0:
         _check(LF_ERR_INVALID)
-    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)  # status words start at zero
 
 
 def lf_attn_fwd(p, q_s, k_s, v_s, q_g, k_g, v_g, mask, o, lse, ws, stream=None):
@@ -235,7 +235,7 @@ def cross_workspace(p, device="cuda"):
     nbytes = lf_attn_cross_workspace_size(p)
     if nbytes == 0:
         _check(LF_ERR_INVALID)
-    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)  # status words start at zero
 
 
 def lf_attn_cross_fwd(p, q, k, v, key_mask, o, lse, ws, stream=None):
@@ -261,7 +261,7 @@ def proj_workspace(p, max_rows: int = 0, device="cuda"):
     nbytes = lf_proj_workspace_size(p, max_rows)
     if nbytes == 0:
         _check(LF_ERR_INVALID)
-    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)  # status words start at zero
 
 
 def lf_proj_in(p, x, w_in, b_in, outs, ws, rows_mask=None, rows_code: int = 2, max_rows: int = 0,

@@ -699,6 +699,8 @@ def main():
                     help="skip the other workloads reported under 'workloads'")
     ap.add_argument("--proj", action="store_true",
                     help="time only the projection GEMMs around the layer (one JSON line)")
+    ap.add_argument("--cross", action="store_true",
+                    help="time only the LED decoder cross-attention (one JSON line)")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
     layout = resolve_world(args.gpus)
@@ -713,6 +715,14 @@ def main():
 
     if args.decode:
         return run_decode(args, wl)
+    if args.cross:
+        cr = cross_numbers(args.steps, args.warmup, torch.device("cuda", 0))
+        print(json.dumps({"metric": "LED decoder cross-attention TFLOP/s (1024 queries x 16384 keys, 16 heads, B 2)",
+                          "value": cr["tflops_step"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+                          "warmup": args.warmup, "ms_per_step": cr["step_us"] * 1e-3, "higher_is_better": True,
+                          "dtype": "bf16", "data": "synthetic", "config": {"workload": "led decoder cross-attention"},
+                          "cross_attention": cr}), flush=True)
+        return 0
     if args.proj:
         pr = projection_numbers(wl, args.steps, args.warmup, torch.device("cuda", 0))
         tot_f = sum(v["flops"] for k, v in pr.items() if isinstance(v, dict) and "flops" in v)

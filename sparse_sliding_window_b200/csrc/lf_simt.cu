@@ -39,6 +39,8 @@ __device__ int lf_mask_scan(const LfDev &P, int b, bool write_tables, int32_t *g
   const int per = (n + 1023) / 1024;
   const int s = tid * per, e = min(n, s + per);
   int c = 0, v = 0, bad = 0, gmin = n, gmax = -1;
+  // unrolled so that several of the thread's loads are in flight at once
+#pragma unroll 8
   for (int i = s; i < e; i++) {
     int x = m[i];
     if (x == 2) {
@@ -57,6 +59,7 @@ __device__ int lf_mask_scan(const LfDev &P, int b, bool write_tables, int32_t *g
   if (bad) atomicOr(&s_bad, 1);
   if (tid == 0) s_total = total;
   int32_t *gr = P.grank + (size_t)b * (n + 1);
+#pragma unroll 8
   for (int i = s; i < e; i++) {
     if (write_tables) gr[i] = off;  // globals before position i
     if (m[i] == 2) {
@@ -632,30 +635,21 @@ cudaError_t lf_launch_simt_bwd(const LfLaunch &L, const void *qs, const void *ks
   }
 }
 
-// delta = rowsum(dO * O) and dK_g / dV_g (every key, over the global rows),
-// shared by the CUDA-core and the tensor-core backward.
+// delta = rowsum(dO * O) alone (the tensor-core backward computes dK_g / dV_g
+// together with dQ_g, in lf_bwd_gkey_kernel)
 template <typename T>
-static cudaError_t lf_bwd_delta_dkvg_t(const LfLaunch &L, const void *o, const void *dO,
-                                       float *delta, const void *qg, const void *kg,
-                                       const void *vg, const float *lse, void *dkg, void *dvg) {
-  long long rows = (long long)L.dev.B * L.dev.H * L.dev.n;
-  const unsigned ggrid = (unsigned)((rows * (LF_HD / LfVec<T>::N) + 255) / 256);  // a lane group per row
-  lf_bwd_delta_kernel<T><<<ggrid, 256, 0, L.stream>>>(L.dev, (const T *)o, (const T *)dO, delta);
-  lf_bwd_dkv_g_kernel<T><<<ggrid, 256, 0, L.stream>>>(L.dev, (const T *)qg, (const T *)kg,
-                                                     (const T *)vg, lse, (const T *)dO, delta,
-                                                     (T *)dkg, (T *)dvg);
-  lf_launches_add(2);
+static cudaError_t lf_bwd_delta_t(const LfLaunch &L, const void *o, const void *dO, float *delta) {
+  const long long rows = (long long)L.dev.B * L.dev.H * L.dev.n;
+  const unsigned grid = (unsigned)((rows * (LF_HD / LfVec<T>::N) + 255) / 256);  // a lane group per row
+  lf_bwd_delta_kernel<T><<<grid, 256, 0, L.stream>>>(L.dev, (const T *)o, (const T *)dO, delta);
+  lf_launches_add(1);
   return cudaGetLastError();
 }
 
-cudaError_t lf_launch_bwd_delta_dkvg(const LfLaunch &L, const void *o, const void *dO, float *delta,
-                                     const void *qg, const void *kg, const void *vg, const float *lse,
-                                     void *dkg, void *dvg) {
-  if (L.dtype == LF_F16)
-    return lf_bwd_delta_dkvg_t<__half>(L, o, dO, delta, qg, kg, vg, lse, dkg, dvg);
-  if (L.dtype == LF_BF16)
-    return lf_bwd_delta_dkvg_t<__nv_bfloat16>(L, o, dO, delta, qg, kg, vg, lse, dkg, dvg);
-  return lf_bwd_delta_dkvg_t<float>(L, o, dO, delta, qg, kg, vg, lse, dkg, dvg);
+cudaError_t lf_launch_bwd_delta(const LfLaunch &L, const void *o, const void *dO, float *delta) {
+  if (L.dtype == LF_F16) return lf_bwd_delta_t<__half>(L, o, dO, delta);
+  if (L.dtype == LF_BF16) return lf_bwd_delta_t<__nv_bfloat16>(L, o, dO, delta);
+  return lf_bwd_delta_t<float>(L, o, dO, delta);
 }
 
 // ============================================================ decode step

@@ -622,77 +622,100 @@ __global__ void __launch_bounds__(32 * LF_BW_RED_WARPS)
   }
 }
 
-// dQ_g of the global rows: every valid key through Q_g / K_g / V_g.  One
-// block per (b, h, global e, chunk of keys), grid-strided, a lane group per
-// key as in lf_bwd_gcol_kernel; partial sums reduced below.
+// dK_g, dV_g of every key and the dQ_g partials of the global rows in one
+// pass over the keys (both need, per key j and global row g, the same
+// p_gj = exp(s_gj - lse_g) and dS_gj = p_gj (dP_gj - D_g) scale): one block
+// per (b, h, chunk of LF_BW_ROWS_PER_CHUNK keys), grid-strided; a lane group
+// (64 / N lanes, 16 bytes each) per key, two keys per group.  Per global
+// row the block's dS_gj k_j are added in a fixed order (the groups of a
+// warp, then the warps) into the chunk's dQ_g partial, which
+// lf_bwd_grow_reduce adds up.  Rows of mask-0 keys are zero.
 template <typename T>
 __global__ void __launch_bounds__(256)
-    lf_bwd_grow_kernel(LfDev P, const T *qg, const T *kg, const T *vg, const float *lse,
-                       const T *dO, const float *delta, float *part, int nch) {
+    lf_bwd_gkey_kernel(LfDev P, const T *qg, const T *kg, const T *vg, const float *lse,
+                       const T *dO, const float *delta, T *dkg, T *dvg, float *part_q, int nch) {
   constexpr int N = LfVec<T>::N, TPR = LF_HD / N, GPB = 256 / TPR;
+  constexpr int KPG = LF_BW_ROWS_PER_CHUNK / GPB;  // keys per group
   __shared__ float s_red[8][LF_HD];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int grp = threadIdx.x / TPR, pi = threadIdx.x % TPR;
-  const long long units = (long long)P.B * P.H * P.G * nch;
+  const int n = P.n;
+  const long long units = (long long)P.B * P.H * nch;
   for (long long un = blockIdx.x; un < units; un += gridDim.x) {
     const int c = (int)(un % nch);
-    const long long be = un / nch;
-    const int e = (int)(be % P.G);
-    const long long bh = be / P.G;
-    const int b = (int)(bh / P.H), n = P.n;
-    const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
-    float aq[N];
+    const long long bh = un / nch;
+    const int b = (int)(bh / P.H);
+    const int32_t *m = P.mask + (size_t)b * n;
+    const size_t base = (size_t)bh * n * LF_HD + pi * N;
+    float kx[KPG][N], vx[KPG][N], ak[KPG][N], av[KPG][N];
+    bool on[KPG];
 #pragma unroll
-    for (int k = 0; k < N; k++) aq[k] = 0.f;
-    if (e < ng) {
-      const int g = P.gidx[(size_t)b * P.G + e];
-      const int32_t *m = P.mask + (size_t)b * n;
-      const size_t base = (size_t)bh * n * LF_HD + pi * N;
+    for (int kk = 0; kk < KPG; kk++) {
+      const int j = c * LF_BW_ROWS_PER_CHUNK + grp + GPB * kk;
+      const int jc = min(j, n - 1);
+      on[kk] = j < n && m[jc] != 0;
+      LfVec<T>::ld(kg + base + (size_t)jc * LF_HD, kx[kk]);
+      LfVec<T>::ld(vg + base + (size_t)jc * LF_HD, vx[kk]);
+#pragma unroll
+      for (int k = 0; k < N; k++) ak[kk][k] = av[kk][k] = 0.f;
+    }
+    const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
+    const int32_t *gl = P.gidx + (size_t)b * P.G;
+    for (int e = 0; e < ng; e++) {
+      const int g = gl[e];
       const size_t gr = (size_t)bh * n + g;
-      float q[N], go[N];
+      float q[N], go[N], aq[N];
       LfVec<T>::ld(qg + base + (size_t)g * LF_HD, q);
       LfVec<T>::ld(dO + base + (size_t)g * LF_HD, go);
       const float L2 = lse[gr] * LF_LOG2E, Dg = delta[gr];
-      const int j0 = c * LF_BW_ROWS_PER_CHUNK, j1 = min(n, j0 + LF_BW_ROWS_PER_CHUNK);
-      for (int rr = 0; rr < LF_BW_ROWS_PER_CHUNK; rr += GPB) {
-        const int j = j0 + rr + grp;
-        const bool valid = j < j1;
-        const int jc = valid ? j : j1 - 1;
-        float kx[N], vx[N];
-        LfVec<T>::ld(kg + base + (size_t)jc * LF_HD, kx);
-        LfVec<T>::ld(vg + base + (size_t)jc * LF_HD, vx);
-        float s = 0.f, dp = 0.f;
+#pragma unroll
+      for (int k = 0; k < N; k++) aq[k] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < KPG; kk++) {
+        float sc = 0.f, dp = 0.f;
 #pragma unroll
         for (int k = 0; k < N; k++) {
-          s += q[k] * kx[k];
-          dp += go[k] * vx[k];
+          sc += q[k] * kx[kk][k];
+          dp += go[k] * vx[kk][k];
         }
-        s = lf_group_sum<TPR>(s);
+        sc = lf_group_sum<TPR>(sc);
         dp = lf_group_sum<TPR>(dp);
-        if (!valid || m[j] == 0) continue;
-        const float pr = exp2f(s * P.scale_log2 - L2);
+        if (!on[kk]) continue;
+        const float pr = exp2f(sc * P.scale_log2 - L2);
         const float ds = pr * (dp - Dg) * P.scale;
 #pragma unroll
-        for (int k = 0; k < N; k++) aq[k] += ds * kx[k];
+        for (int k = 0; k < N; k++) {
+          ak[kk][k] += ds * q[k];
+          av[kk][k] += pr * go[k];
+          aq[k] += ds * kx[kk][k];
+        }
       }
+      // this chunk's dQ_g partial of global row e
+#pragma unroll
+      for (int o = TPR; o < 32; o <<= 1)
+#pragma unroll
+        for (int k = 0; k < N; k++) aq[k] += __shfl_xor_sync(0xffffffffu, aq[k], o);
+      if (lane < TPR)
+#pragma unroll
+        for (int k = 0; k < N; k++) s_red[warp][pi * N + k] = aq[k];
+      __syncthreads();
+      if (warp == 0) {
+        float *dst = part_q + (((size_t)bh * P.G + e) * nch + c) * LF_HD;
+        for (int x = lane; x < LF_HD; x += 32) {
+          float t = 0.f;
+          for (int w = 0; w < 8; w++) t += s_red[w][x];
+          dst[x] = t;
+        }
+      }
+      __syncthreads();
     }
 #pragma unroll
-    for (int o = TPR; o < 32; o <<= 1)
-#pragma unroll
-      for (int k = 0; k < N; k++) aq[k] += __shfl_xor_sync(0xffffffffu, aq[k], o);
-    if (lane < TPR)
-#pragma unroll
-      for (int k = 0; k < N; k++) s_red[warp][pi * N + k] = aq[k];
-    __syncthreads();
-    if (warp == 0) {
-      float *dst = part + (size_t)un * LF_HD;
-      for (int x = lane; x < LF_HD; x += 32) {
-        float t = 0.f;
-        for (int w = 0; w < 8; w++) t += s_red[w][x];
-        dst[x] = t;
-      }
+    for (int kk = 0; kk < KPG; kk++) {
+      const int j = c * LF_BW_ROWS_PER_CHUNK + grp + GPB * kk;
+      if (j >= n) continue;
+      LfVec<T>::st(dkg + base + (size_t)j * LF_HD, ak[kk]);
+      LfVec<T>::st(dvg + base + (size_t)j * LF_HD, av[kk]);
     }
-    __syncthreads();
   }
 }
 
@@ -756,25 +779,38 @@ static cudaError_t lf_bwd_global_parts(const LfLaunch &L, const LfTcBwdArgs &a, 
     const unsigned rgrid = (unsigned)std::min<long long>(wr, 4096);
     lf_bwd_gcol_reduce<T><<<rgrid, 32 * LF_BW_RED_WARPS, 0, L.stream>>>(D, part_kv, nch, (T *)a.dks,
                                                                         (T *)a.dvs);
-    lf_bwd_grow_kernel<T><<<ugrid, 256, 0, L.stream>>>(
-        D, (const T *)a.qg, (const T *)a.kg, (const T *)a.vg, a.lse, (const T *)a.dO, delta, part_q, nch);
     lf_bwd_grow_reduce<T><<<rgrid, 32 * LF_BW_RED_WARPS, 0, L.stream>>>(D, part_q, nch, (T *)a.dqg);
-    lf_launches_add(4);
+    lf_launches_add(3);
   }
   return cudaGetLastError();
 }
 
-cudaError_t lf_launch_bwd_delta_dkvg(const LfLaunch &L, const void *o, const void *dO, float *delta,
-                                     const void *qg, const void *kg, const void *vg, const float *lse,
-                                     void *dkg, void *dvg);
+cudaError_t lf_launch_bwd_delta(const LfLaunch &L, const void *o, const void *dO, float *delta);
 
 int lf_tc_bwd(const LfLaunch &L, const LfTcBwdArgs &a, char *err, size_t errlen) {
   const LfDev &D = L.dev;
   const int f16 = L.dtype == LF_F16 ? 1 : 0;
   float *delta = (float *)(L.ws_base + L.ws.delta);
   cudaError_t ce;
-  // delta = rowsum(dO * O); dK_g, dV_g (every key, over the global rows)
-  ce = lf_launch_bwd_delta_dkvg(L, a.o, a.dO, delta, a.qg, a.kg, a.vg, a.lse, a.dkg, a.dvg);
+  // delta = rowsum(dO * O); then dK_g, dV_g of every key and the dQ_g
+  // partials, in one pass over the keys
+  const int nch = (D.n + LF_BW_ROWS_PER_CHUNK - 1) / LF_BW_ROWS_PER_CHUNK;
+  float *part_kv = (float *)(L.ws_base + L.ws.part_acc), *part_q = (float *)(L.ws_base + L.ws.part_ml);
+  ce = lf_launch_bwd_delta(L, a.o, a.dO, delta);
+  if (ce == cudaSuccess) {
+    const unsigned kgrid = (unsigned)std::min<long long>((long long)D.B * D.H * nch, 148LL * 16);
+    if (f16)
+      lf_bwd_gkey_kernel<__half><<<kgrid, 256, 0, L.stream>>>(
+          D, (const __half *)a.qg, (const __half *)a.kg, (const __half *)a.vg, a.lse,
+          (const __half *)a.dO, delta, (__half *)a.dkg, (__half *)a.dvg, part_q, nch);
+    else
+      lf_bwd_gkey_kernel<__nv_bfloat16><<<kgrid, 256, 0, L.stream>>>(
+          D, (const __nv_bfloat16 *)a.qg, (const __nv_bfloat16 *)a.kg, (const __nv_bfloat16 *)a.vg,
+          a.lse, (const __nv_bfloat16 *)a.dO, delta, (__nv_bfloat16 *)a.dkg, (__nv_bfloat16 *)a.dvg,
+          part_q, nch);
+    lf_launches_add(1);
+    ce = cudaGetLastError();
+  }
   if (ce != cudaSuccess) {
     snprintf(err, errlen, "backward delta / dK_g launch: %s", cudaGetErrorString(ce));
     return LF_ERR_CUDA;
@@ -864,8 +900,6 @@ int lf_tc_bwd(const LfLaunch &L, const LfTcBwdArgs &a, char *err, size_t errlen)
     }
   }
   // global-column part of dK_s / dV_s (after the band part) and dQ_g
-  const int nch = (D.n + LF_BW_ROWS_PER_CHUNK - 1) / LF_BW_ROWS_PER_CHUNK;
-  float *part_kv = (float *)(L.ws_base + L.ws.part_acc), *part_q = (float *)(L.ws_base + L.ws.part_ml);
   ce = f16 ? lf_bwd_global_parts<__half>(L, a, delta, part_kv, part_q, nch)
            : lf_bwd_global_parts<__nv_bfloat16>(L, a, delta, part_kv, part_q, nch);
   if (ce != cudaSuccess) {

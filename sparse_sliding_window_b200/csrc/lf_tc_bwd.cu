@@ -51,7 +51,8 @@
 #define LF_BW_BK 64  // columns (keys / queries) per column tile
 #define LF_BW_MAX_MAPS 192  // kernel parameters may take up to 32 KB
 #define LF_BW_MAX_SEG 96
-#define LF_BW_ROWS_PER_CHUNK 64  // rows (keys) per warp of the global-row / -column parts
+#define LF_BW_ROWS_PER_CHUNK 64  // keys per chunk of the global-key pass (dK_g, dV_g, dQ_g)
+#define LF_BW_GCOL_ROWS 256      // rows per chunk of the global-column pass
 
 #define LF_BW_R0 0
 #define LF_BW_R1 16384
@@ -482,7 +483,7 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 2)
 // Global-column part of dK_s / dV_s: a global key g is attended by every
 // local row, by its window or by its global column (union); the band kernel
 // covered the window, this pass the rows whose window misses g.  One block of
-// 256 threads per (b, h, global e, chunk of LF_BW_ROWS_PER_CHUNK rows),
+// 256 threads per (b, h, global e, chunk of LF_BW_GCOL_ROWS rows),
 // grid-strided: a lane group (64 / N lanes, 16 bytes of a row each) per row,
 // the groups' sums added in a fixed order into the chunk's partial, which
 // lf_bwd_gcol_reduce adds up.
@@ -512,8 +513,9 @@ __global__ void __launch_bounds__(256)
       float kx[N], vx[N];
       LfVec<T>::ld(ks + base + (size_t)g * LF_HD, kx);
       LfVec<T>::ld(vs + base + (size_t)g * LF_HD, vx);
-      const int i0 = c * LF_BW_ROWS_PER_CHUNK, i1 = min(n, i0 + LF_BW_ROWS_PER_CHUNK);
-      for (int rr = 0; rr < LF_BW_ROWS_PER_CHUNK; rr += GPB) {
+      const int i0 = c * LF_BW_GCOL_ROWS, i1 = min(n, i0 + LF_BW_GCOL_ROWS);
+#pragma unroll 4
+      for (int rr = 0; rr < LF_BW_GCOL_ROWS; rr += GPB) {
         const int i = i0 + rr + grp;
         const bool valid = i < i1;
         const int ic = valid ? i : i1 - 1;
@@ -766,18 +768,19 @@ __global__ void __launch_bounds__(32 * LF_BW_RED_WARPS)
 template <typename T>
 static cudaError_t lf_bwd_global_parts(const LfLaunch &L, const LfTcBwdArgs &a, const float *delta,
                                        float *part_kv, float *part_q, int nch) {
+  const int nchc = (L.dev.n + LF_BW_GCOL_ROWS - 1) / LF_BW_GCOL_ROWS;  // global-column chunks
   const LfDev &D = L.dev;
   cudaError_t e;
   // dQ_g: zero rows outside the global tokens, then the global rows
   e = cudaMemsetAsync(a.dqg, 0, (size_t)D.B * D.H * D.n * LF_HD * sizeof(T), L.stream);
   if (e != cudaSuccess) return e;
   if (D.G > 0) {
-    const long long wk = (long long)D.B * D.H * D.G * nch, wr = (long long)D.B * D.H * D.G;
+    const long long wk = (long long)D.B * D.H * D.G * nchc, wr = (long long)D.B * D.H * D.G;
     const unsigned ugrid = (unsigned)std::min<long long>(wk, 148LL * 16);  // grid-strided units
     lf_bwd_gcol_kernel<T><<<ugrid, 256, 0, L.stream>>>(
-        D, (const T *)a.qs, (const T *)a.ks, (const T *)a.vs, a.lse, (const T *)a.dO, delta, part_kv, nch);
+        D, (const T *)a.qs, (const T *)a.ks, (const T *)a.vs, a.lse, (const T *)a.dO, delta, part_kv, nchc);
     const unsigned rgrid = (unsigned)std::min<long long>(wr, 4096);
-    lf_bwd_gcol_reduce<T><<<rgrid, 32 * LF_BW_RED_WARPS, 0, L.stream>>>(D, part_kv, nch, (T *)a.dks,
+    lf_bwd_gcol_reduce<T><<<rgrid, 32 * LF_BW_RED_WARPS, 0, L.stream>>>(D, part_kv, nchc, (T *)a.dks,
                                                                         (T *)a.dvs);
     lf_bwd_grow_reduce<T><<<rgrid, 32 * LF_BW_RED_WARPS, 0, L.stream>>>(D, part_q, nch, (T *)a.dqg);
     lf_launches_add(3);

@@ -120,17 +120,28 @@ __global__ void __launch_bounds__(1024)
   if (tables)  // the global list itself, as the mask pass writes it
     for (int e = threadIdx.x; e < ng; e += blockDim.x) P.gidx[(size_t)b * P.G + e] = s_gl[e];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = warp; e < Gka; e += 32) {
-    uint32_t q = 0, k = 0, v = 0;
-    if (e < ng) {
-      const size_t src = ((size_t)bh * P.n + s_gl[e]) * LF_HD + 2 * lane;
-      q = *reinterpret_cast<const uint32_t *>(qg + src);
-      k = *reinterpret_cast<const uint32_t *>(ks + src);
-      v = *reinterpret_cast<const uint32_t *>(vs + src);
+  // four rows per warp per round, every load of a round issued before its stores
+  for (int e0 = warp; e0 < Gka; e0 += 4 * 32) {
+    uint32_t q[4], k[4], v[4];
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+      const int e = e0 + 32 * u;
+      q[u] = k[u] = v[u] = 0;
+      if (e < ng) {
+        const size_t src = ((size_t)bh * P.n + s_gl[e]) * LF_HD + 2 * lane;
+        q[u] = *reinterpret_cast<const uint32_t *>(qg + src);
+        k[u] = *reinterpret_cast<const uint32_t *>(ks + src);
+        v[u] = *reinterpret_cast<const uint32_t *>(vs + src);
+      }
     }
-    if (e < Ga) *reinterpret_cast<uint32_t *>(qg_c + ((size_t)bh * Ga + e) * LF_HD + 2 * lane) = q;
-    *reinterpret_cast<uint32_t *>(ks_c + ((size_t)bh * Gka + e) * LF_HD + 2 * lane) = k;
-    *reinterpret_cast<uint32_t *>(vs_c + ((size_t)bh * Gka + e) * LF_HD + 2 * lane) = v;
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+      const int e = e0 + 32 * u;
+      if (e >= Gka) break;
+      if (e < Ga) *reinterpret_cast<uint32_t *>(qg_c + ((size_t)bh * Ga + e) * LF_HD + 2 * lane) = q[u];
+      *reinterpret_cast<uint32_t *>(ks_c + ((size_t)bh * Gka + e) * LF_HD + 2 * lane) = k[u];
+      *reinterpret_cast<uint32_t *>(vs_c + ((size_t)bh * Gka + e) * LF_HD + 2 * lane) = v[u];
+    }
   }
 }
 

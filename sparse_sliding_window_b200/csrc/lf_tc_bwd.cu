@@ -378,27 +378,37 @@ __device__ __forceinline__ void lf_tc_bwd_item(const LfBwParams &P, int item, ui
       for (int cc = 0; cc < NC; cc++) {
         uint32_t ds_w[16], p_w[16];
         if (__any_sync(0xffffffffu, w[cc] != 0u)) {
-          float x[32], y[32];
-          lf_tmem_ld32(tS + 32 * cc, x);
-          lf_tmem_ld32(tDP + 32 * cc, y);
+          // S and dP of the chunk in flight together, one wait
+          uint32_t x[32], y[32];
+          lf_tmem_ld32_nowait(tS + 32 * cc, x);
+          lf_tmem_ld32_nowait(tDP + 32 * cc, y);
+          lf_tmem_wait_ld_regs(x);
+          lf_tmem_pin_regs(y);
           const uint32_t wc = w[cc];
 #pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            float p0 = 0.f, p1 = 0.f, g0 = 0.f, g1 = 0.f;
-            const float l0 = kModeQ ? lse2 : clse2[32 * cc + k];
-            const float l1 = kModeQ ? lse2 : clse2[32 * cc + k + 1];
-            const float d0 = kModeQ ? dd : cdd[32 * cc + k];
-            const float d1 = kModeQ ? dd : cdd[32 * cc + k + 1];
-            if ((wc >> k) & 1u) {
-              p0 = lf_ex2(fmaf(x[k], sl2, -l0));
-              g0 = p0 * (y[k] - d0) * scale;
+          for (int k4 = 0; k4 < 32; k4 += 4) {
+            // the columns' log-normalisers and D (mode KV), four per shared-memory load
+            float4 l4 = make_float4(lse2, lse2, lse2, lse2), d4 = make_float4(dd, dd, dd, dd);
+            if (!kModeQ) {
+              l4 = *reinterpret_cast<const float4 *>(clse2 + 32 * cc + k4);
+              d4 = *reinterpret_cast<const float4 *>(cdd + 32 * cc + k4);
             }
-            if ((wc >> (k + 1)) & 1u) {
-              p1 = lf_ex2(fmaf(x[k + 1], sl2, -l1));
-              g1 = p1 * (y[k + 1] - d1) * scale;
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+            for (int u = 0; u < 4; u += 2) {
+              const int k = k4 + u;
+              float p0 = 0.f, p1 = 0.f, g0 = 0.f, g1 = 0.f;
+              if ((wc >> k) & 1u) {
+                p0 = lf_ex2(fmaf(__uint_as_float(x[k]), sl2, -lv[u]));
+                g0 = p0 * (__uint_as_float(y[k]) - dv[u]) * scale;
+              }
+              if ((wc >> (k + 1)) & 1u) {
+                p1 = lf_ex2(fmaf(__uint_as_float(x[k + 1]), sl2, -lv[u + 1]));
+                g1 = p1 * (__uint_as_float(y[k + 1]) - dv[u + 1]) * scale;
+              }
+              ds_w[k / 2] = lf_pack2<kF16>(g0, g1);
+              p_w[k / 2] = lf_pack2<kF16>(p0, p1);
             }
-            ds_w[k / 2] = lf_pack2<kF16>(g0, g1);
-            p_w[k / 2] = lf_pack2<kF16>(p0, p1);
           }
         } else {
 #pragma unroll

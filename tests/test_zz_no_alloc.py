@@ -8,8 +8,8 @@ that a problem too large for the array is refused up front.
 
 The array also holds the call's device status word, read through
 lf_attn_status_noalloc: a mask value outside {0, 1, 2} must come back as
-LF_ERR_DEVICE_INPUT there, and the next good call must come back clean (each
-call clears the word).  Free device memory is compared around the calls: the
+LF_ERR_DEVICE_INPUT there (the read clears the word), and the next good call
+must come back clean.  Free device memory is compared around the calls: the
 entry point exists so that nothing is allocated, so it must not drop.
 
 Collected last on purpose (file name), so a run that stops at the first

@@ -219,14 +219,14 @@ int lf_attn_set_test_hooks(uint32_t wait_limit_us, int skip_kv_tile);
  * the library's device image, which every GPU that loads the library holds
  * until the process exits.  Problems whose lf_attn_workspace_size exceeds it
  * are rejected with LF_ERR_UNSUPPORTED (use lf_attn_fwd).  The call allocates
- * nothing.  Its first call on a device looks up the array's device address
- * (with that device current; `stream` must belong to it); make that first
- * call before any stream capture.  All calls on a device share the one
- * array, so calls that may overlap on the GPU (other streams, other host
- * threads) race and must be serialised by the caller.  The device status
- * word of this variant lives in that array: read it with
- * lf_attn_status_noalloc.  The cached address does not survive a
- * cudaDeviceReset of the device; do not use this call after one. */
+ * nothing.  Every call looks up the array's device address on the current
+ * device (`stream` must belong to it; a symbol lookup, no allocation, so a
+ * context torn down and created again is followed); make the first call on
+ * a device before any stream capture, since it may load the library's
+ * device code.  All calls on a device share the one array, so calls that
+ * may overlap on the GPU (other streams, other host threads) race and must
+ * be serialised by the caller.  The device status word of this variant
+ * lives in that array: read it with lf_attn_status_noalloc. */
 int lf_attn_fwd_noalloc(const lf_attn_params *p, const void *q_s,
                         const void *k_s, const void *v_s, const void *q_g,
                         const void *k_g, const void *v_g, const int32_t *mask,

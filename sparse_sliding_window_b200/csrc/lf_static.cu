@@ -12,51 +12,28 @@
 //
 // On the host, the array's name is only a host-side stand-in for the device
 // symbol, never a device address; the device address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress with the caller's device current, on every call (a
+// lookup, no allocation), so nothing goes stale when a context is torn down
+// and created again.
 #include <stdio.h>
-
-#include <mutex>
 
 #include "lf_attn.h"
 
-#define LF_STATIC_MAX_DEVICES 64
-
 static __device__ __align__(256) unsigned char lf_static_ws[LF_STATIC_WORKSPACE_BYTES];
-
-static std::mutex g_static_mu;
-static void *g_static_addr[LF_STATIC_MAX_DEVICES];
 
 // defined in lf_api.cu: record an error for lf_attn_last_error()
 int lf_record_error(int code, const char *msg);
 
-// Device address of the static scratch on the current device; looked up
-// once per device (with that device current) and cached.
+// Device address of the static scratch on the current device.
 static int lf_static_base(void **base, const char *who) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) {
-    char msg[128];
-    snprintf(msg, sizeof(msg), "%s: cudaGetDevice failed", who);
+  void *ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, lf_static_ws);
+  if (e != cudaSuccess || !ptr) {
+    char msg[160];
+    snprintf(msg, sizeof(msg), "%s: cudaGetSymbolAddress failed (%s)", who, cudaGetErrorString(e));
     return lf_record_error(LF_ERR_CUDA, msg);
   }
-  if (dev < 0 || dev >= LF_STATIC_MAX_DEVICES) {
-    char msg[128];
-    snprintf(msg, sizeof(msg), "%s: device ordinal out of range", who);
-    return lf_record_error(LF_ERR_UNSUPPORTED, msg);
-  }
-  std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_addr[dev]) {
-    // first use on this device (the current one): look the symbol up
-    void *ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, lf_static_ws);
-    if (e != cudaSuccess || !ptr) {
-      char msg[128];
-      snprintf(msg, sizeof(msg), "%s: cudaGetSymbolAddress failed", who);
-      return lf_record_error(LF_ERR_CUDA, msg);
-    }
-    g_static_addr[dev] = ptr;
-  }
-  *base = g_static_addr[dev];
+  *base = ptr;
   return LF_OK;
 }
 

@@ -529,9 +529,13 @@ __global__ void __launch_bounds__(256)
         const int i = i0 + rr + grp;
         const bool valid = i < i1;
         const int ic = valid ? i : i1 - 1;
+        // every load of the row issued together (none waits on the mask test)
         float q[N], go[N];
         LfVec<T>::ld(qs + base + (size_t)ic * LF_HD, q);
         LfVec<T>::ld(dO + base + (size_t)ic * LF_HD, go);
+        const size_t ir = (size_t)bh * n + ic;
+        const int mi = m[ic];
+        const float lse_i = lse[ir], dl_i = delta[ir];
         float s = 0.f, dp = 0.f;
 #pragma unroll
         for (int k = 0; k < N; k++) {
@@ -540,10 +544,9 @@ __global__ void __launch_bounds__(256)
         }
         s = lf_group_sum<TPR>(s);
         dp = lf_group_sum<TPR>(dp);
-        if (!valid || m[i] != 1 || lf_in_window(i, g, P.r, d, P.causal)) continue;
-        const size_t ir = (size_t)bh * n + i;
-        const float pr = exp2f(s * P.scale_log2 - lse[ir] * LF_LOG2E);
-        const float ds = pr * (dp - delta[ir]) * P.scale;
+        if (!valid || mi != 1 || lf_in_window(i, g, P.r, d, P.causal)) continue;
+        const float pr = exp2f(s * P.scale_log2 - lse_i * LF_LOG2E);
+        const float ds = pr * (dp - dl_i) * P.scale;
 #pragma unroll
         for (int k = 0; k < N; k++) {
           ak[k] += ds * q[k];
@@ -661,6 +664,10 @@ __global__ void __launch_bounds__(256)
     const size_t base = (size_t)bh * n * LF_HD + pi * N;
     float kx[KPG][N], vx[KPG][N], ak[KPG][N], av[KPG][N];
     bool on[KPG];
+    // the sequence's global count and first global row, read while the keys load
+    const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
+    const int32_t *gl = P.gidx + (size_t)b * P.G;
+    int g_next = P.G > 0 ? gl[0] : 0;  // (the list has G >= 1 entries when G > 0)
 #pragma unroll
     for (int kk = 0; kk < KPG; kk++) {
       const int j = c * LF_BW_ROWS_PER_CHUNK + grp + GPB * kk;
@@ -671,10 +678,9 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
       for (int k = 0; k < N; k++) ak[kk][k] = av[kk][k] = 0.f;
     }
-    const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
-    const int32_t *gl = P.gidx + (size_t)b * P.G;
     for (int e = 0; e < ng; e++) {
-      const int g = gl[e];
+      const int g = g_next;
+      if (e + 1 < ng) g_next = gl[e + 1];
       const size_t gr = (size_t)bh * n + g;
       float q[N], go[N], aq[N];
       LfVec<T>::ld(qg + base + (size_t)g * LF_HD, q);

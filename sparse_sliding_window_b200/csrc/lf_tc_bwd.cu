@@ -498,7 +498,7 @@ __global__ void __launch_bounds__(LF_BW_THREADS, 2)
 // the groups' sums added in a fixed order into the chunk's partial, which
 // lf_bwd_gcol_reduce adds up.
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
     lf_bwd_gcol_kernel(LfDev P, const T *qs, const T *ks, const T *vs, const float *lse,
                        const T *dO, const float *delta, float *part, int nch) {
   constexpr int N = LfVec<T>::N, TPR = LF_HD / N, GPB = 256 / TPR;
@@ -524,33 +524,41 @@ __global__ void __launch_bounds__(256)
       LfVec<T>::ld(ks + base + (size_t)g * LF_HD, kx);
       LfVec<T>::ld(vs + base + (size_t)g * LF_HD, vx);
       const int i0 = c * LF_BW_GCOL_ROWS, i1 = min(n, i0 + LF_BW_GCOL_ROWS);
-#pragma unroll 4
-      for (int rr = 0; rr < LF_BW_GCOL_ROWS; rr += GPB) {
-        const int i = i0 + rr + grp;
-        const bool valid = i < i1;
-        const int ic = valid ? i : i1 - 1;
-        // every load of the row issued together (none waits on the mask test)
-        float q[N], go[N];
-        LfVec<T>::ld(qs + base + (size_t)ic * LF_HD, q);
-        LfVec<T>::ld(dO + base + (size_t)ic * LF_HD, go);
-        const size_t ir = (size_t)bh * n + ic;
-        const int mi = m[ic];
-        const float lse_i = lse[ir], dl_i = delta[ir];
-        float s = 0.f, dp = 0.f;
+      // four row groups per round: every load of the round is issued before
+      // any of its arithmetic (none waits on a mask test)
+      for (int rr = 0; rr < LF_BW_GCOL_ROWS; rr += 4 * GPB) {
+        float q[4][N], go[4][N], lse_i[4], dl_i[4];
+        int mi[4];
 #pragma unroll
-        for (int k = 0; k < N; k++) {
-          s += q[k] * kx[k];
-          dp += go[k] * vx[k];
+        for (int u = 0; u < 4; u++) {
+          const int i = i0 + rr + u * GPB + grp;
+          const int ic = i < i1 ? i : i1 - 1;
+          LfVec<T>::ld(qs + base + (size_t)ic * LF_HD, q[u]);
+          LfVec<T>::ld(dO + base + (size_t)ic * LF_HD, go[u]);
+          const size_t ir = (size_t)bh * n + ic;
+          mi[u] = m[ic];
+          lse_i[u] = lse[ir];
+          dl_i[u] = delta[ir];
         }
-        s = lf_group_sum<TPR>(s);
-        dp = lf_group_sum<TPR>(dp);
-        if (!valid || mi != 1 || lf_in_window(i, g, P.r, d, P.causal)) continue;
-        const float pr = exp2f(s * P.scale_log2 - lse_i * LF_LOG2E);
-        const float ds = pr * (dp - dl_i) * P.scale;
 #pragma unroll
-        for (int k = 0; k < N; k++) {
-          ak[k] += ds * q[k];
-          av[k] += pr * go[k];
+        for (int u = 0; u < 4; u++) {
+          const int i = i0 + rr + u * GPB + grp;
+          float s = 0.f, dp = 0.f;
+#pragma unroll
+          for (int k = 0; k < N; k++) {
+            s += q[u][k] * kx[k];
+            dp += go[u][k] * vx[k];
+          }
+          s = lf_group_sum<TPR>(s);
+          dp = lf_group_sum<TPR>(dp);
+          if (i >= i1 || mi[u] != 1 || lf_in_window(i, g, P.r, d, P.causal)) continue;
+          const float pr = exp2f(s * P.scale_log2 - lse_i[u] * LF_LOG2E);
+          const float ds = pr * (dp - dl_i[u]) * P.scale;
+#pragma unroll
+          for (int k = 0; k < N; k++) {
+            ak[k] += ds * q[u][k];
+            av[k] += pr * go[u][k];
+          }
         }
       }
     }

@@ -298,11 +298,19 @@ struct LfRowAcc {
   float q[64];
   float mx, l, a0, a1;
   int self;  // this warp's own row (a valid address for lanes without a key)
-  __device__ __forceinline__ void batch(const T *K, const T *V, size_t base, int j, bool ok, int lane) {
+  // j is the lane's key when `inr` (a row of the sequence); the key counts
+  // when also `cond` and its mask word is nonzero (m == nullptr: no mask).  The key row is loaded
+  // together with the mask word (a row that turns out masked is loaded for
+  // nothing), so a batch waits for one load latency before its scores.
+  __device__ __forceinline__ void batch(const T *K, const T *V, size_t base, const int32_t *m, int j,
+                                        bool inr, bool cond, int lane) {
+    const int jl = inr ? j : self;
+    float k[64];
+    lf_load_row64<T>(K + base + (size_t)jl * LF_HD, k);
+    const bool ok = inr && cond && (!m || m[jl] != 0);
+    j = jl;
     float s = -INFINITY;
     if (ok) {
-      float k[64];
-      lf_load_row64<T>(K + base + (size_t)j * LF_HD, k);
       float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
 #pragma unroll
       for (int c = 0; c < 64; c += 4) {
@@ -373,21 +381,21 @@ __global__ void __launch_bounds__(256, 1)
   if (glob) {
     for (int j0 = 0; j0 < n; j0 += 32) {
       const int j = j0 + lane;
-      st.batch(K, V, base, j, j < n && m[j] != 0, lane);
+      st.batch(K, V, base, m, j, j < n, true, lane);
     }
   } else {
     // window keys j = i + k*d, k in [-r, khi], then the global keys outside it
     const int khi = P.causal ? 0 : P.r;
     for (int k0 = -P.r; k0 <= khi; k0 += 32) {
       const int k = k0 + lane, j = i + k * d;
-      st.batch(K, V, base, j, k <= khi && j >= 0 && j < n && m[j] != 0, lane);
+      st.batch(K, V, base, m, j, k <= khi && j >= 0 && j < n, true, lane);
     }
     const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
     const int32_t *gl = P.gidx + (size_t)b * P.G;
     for (int t0 = 0; t0 < ng; t0 += 32) {
       const int t = t0 + lane;
       const int g = t < ng ? gl[t] : 0;
-      st.batch(K, V, base, g, t < ng && !lf_in_window(i, g, P.r, d, P.causal), lane);
+      st.batch(K, V, base, m, g, t < ng, !lf_in_window(i, g, P.r, d, P.causal), lane);
     }
   }
   const float inv = 1.f / st.l;
@@ -703,7 +711,7 @@ __global__ void __cluster_dims__(LF_DEC_CL, 1, 1) __launch_bounds__(128)
     st.self = t;
     for (int k0 = (crank * 4 + warp) * 32; k0 <= kmax; k0 += 4 * LF_DEC_CL * 32) {
       const int k = k0 + lane;
-      st.batch(kc, vc, base, t - k * d, k <= kmax, lane);
+      st.batch(kc, vc, base, nullptr, t - k * d, k <= kmax, true, lane);
     }
   }
   if (lane == 0) {

@@ -52,6 +52,7 @@
 #define LF_BW_MAX_MAPS 192  // kernel parameters may take up to 32 KB
 #define LF_BW_MAX_SEG 96
 #define LF_BW_ROWS_PER_CHUNK 64  // keys per chunk of the global-key pass (dK_g, dV_g, dQ_g)
+#define LF_BW_GKEY_EB 4          // global rows per reduction of the global-key pass (256 / 64 outputs)
 #define LF_BW_GCOL_ROWS 256      // rows per chunk of the global-column pass
 
 #define LF_BW_R0 0
@@ -659,7 +660,7 @@ __global__ void __launch_bounds__(256)
                        const T *dO, const float *delta, T *dkg, T *dvg, float *part_q, int nch) {
   constexpr int N = LfVec<T>::N, TPR = LF_HD / N, GPB = 256 / TPR;
   constexpr int KPG = LF_BW_ROWS_PER_CHUNK / GPB;  // keys per group
-  __shared__ float s_red[8][LF_HD];
+  __shared__ float s_red[8][LF_BW_GKEY_EB][LF_HD];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int grp = threadIdx.x / TPR, pi = threadIdx.x % TPR;
   const int n = P.n;
@@ -686,51 +687,67 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
       for (int k = 0; k < N; k++) ak[kk][k] = av[kk][k] = 0.f;
     }
-    for (int e = 0; e < ng; e++) {
-      const int g = g_next;
-      if (e + 1 < ng) g_next = gl[e + 1];
-      const size_t gr = (size_t)bh * n + g;
-      float q[N], go[N], aq[N];
-      LfVec<T>::ld(qg + base + (size_t)g * LF_HD, q);
-      LfVec<T>::ld(dO + base + (size_t)g * LF_HD, go);
-      const float L2 = lse[gr] * LF_LOG2E, Dg = delta[gr];
+    // global rows LF_BW_GKEY_EB at a time: their dQ_g partials are reduced
+    // over the block together (two barriers per batch, not per row)
+    for (int e0 = 0; e0 < ng; e0 += LF_BW_GKEY_EB) {
+      const int nb = min(LF_BW_GKEY_EB, ng - e0);  // (block-uniform)
+      float aq[LF_BW_GKEY_EB][N];
 #pragma unroll
-      for (int k = 0; k < N; k++) aq[k] = 0.f;
+      for (int u = 0; u < LF_BW_GKEY_EB; u++)
 #pragma unroll
-      for (int kk = 0; kk < KPG; kk++) {
-        float sc = 0.f, dp = 0.f;
+        for (int k = 0; k < N; k++) aq[u][k] = 0.f;
 #pragma unroll
-        for (int k = 0; k < N; k++) {
-          sc += q[k] * kx[kk][k];
-          dp += go[k] * vx[kk][k];
-        }
-        sc = lf_group_sum<TPR>(sc);
-        dp = lf_group_sum<TPR>(dp);
-        if (!on[kk]) continue;
-        const float pr = exp2f(sc * P.scale_log2 - L2);
-        const float ds = pr * (dp - Dg) * P.scale;
+      for (int u = 0; u < LF_BW_GKEY_EB; u++) {
+        if (u >= nb) break;
+        const int e = e0 + u;
+        const int g = g_next;
+        if (e + 1 < ng) g_next = gl[e + 1];
+        const size_t gr = (size_t)bh * n + g;
+        float q[N], go[N];
+        LfVec<T>::ld(qg + base + (size_t)g * LF_HD, q);
+        LfVec<T>::ld(dO + base + (size_t)g * LF_HD, go);
+        const float L2 = lse[gr] * LF_LOG2E, Dg = delta[gr];
 #pragma unroll
-        for (int k = 0; k < N; k++) {
-          ak[kk][k] += ds * q[k];
-          av[kk][k] += pr * go[k];
-          aq[k] += ds * kx[kk][k];
+        for (int kk = 0; kk < KPG; kk++) {
+          float sc = 0.f, dp = 0.f;
+#pragma unroll
+          for (int k = 0; k < N; k++) {
+            sc += q[k] * kx[kk][k];
+            dp += go[k] * vx[kk][k];
+          }
+          sc = lf_group_sum<TPR>(sc);
+          dp = lf_group_sum<TPR>(dp);
+          if (!on[kk]) continue;
+          const float pr = exp2f(sc * P.scale_log2 - L2);
+          const float ds = pr * (dp - Dg) * P.scale;
+#pragma unroll
+          for (int k = 0; k < N; k++) {
+            ak[kk][k] += ds * q[k];
+            av[kk][k] += pr * go[k];
+            aq[u][k] += ds * kx[kk][k];
+          }
         }
       }
-      // this chunk's dQ_g partial of global row e
+      // this chunk's dQ_g partials of the batch's rows: the groups of a warp,
+      // then the warps in order
 #pragma unroll
-      for (int o = TPR; o < 32; o <<= 1)
+      for (int u = 0; u < LF_BW_GKEY_EB; u++) {
+        if (u >= nb) break;
 #pragma unroll
-        for (int k = 0; k < N; k++) aq[k] += __shfl_xor_sync(0xffffffffu, aq[k], o);
-      if (lane < TPR)
+        for (int o = TPR; o < 32; o <<= 1)
 #pragma unroll
-        for (int k = 0; k < N; k++) s_red[warp][pi * N + k] = aq[k];
+          for (int k = 0; k < N; k++) aq[u][k] += __shfl_xor_sync(0xffffffffu, aq[u][k], o);
+        if (lane < TPR)
+#pragma unroll
+          for (int k = 0; k < N; k++) s_red[warp][u][pi * N + k] = aq[u][k];
+      }
       __syncthreads();
-      if (warp == 0) {
-        float *dst = part_q + (((size_t)bh * P.G + e) * nch + c) * LF_HD;
-        for (int x = lane; x < LF_HD; x += 32) {
+      {
+        const int u = threadIdx.x / LF_HD, x = threadIdx.x % LF_HD;
+        if (u < nb) {
           float t = 0.f;
-          for (int w = 0; w < 8; w++) t += s_red[w][x];
-          dst[x] = t;
+          for (int w = 0; w < 8; w++) t += s_red[w][u][x];
+          part_q[(((size_t)bh * P.G + (e0 + u)) * nch + c) * LF_HD + x] = t;
         }
       }
       __syncthreads();

@@ -590,6 +590,121 @@ __global__ void __launch_bounds__(256, 2)
   }
 }
 
+// The same for sequences with several global keys: one block per (b, h,
+// group of LF_BW_GCOL_E global keys, chunk of LF_BW_GCOL_ROWS rows), every
+// row read once for the group's keys (kept in shared memory, fp32), one
+// partial per key in the same fixed order.
+#define LF_BW_GCOL_E 4
+template <typename T>
+__global__ void __launch_bounds__(256, 2)
+    lf_bwd_gcol4_kernel(LfDev P, const T *qs, const T *ks, const T *vs, const float *lse,
+                        const T *dO, const float *delta, float *part, int nch) {
+  constexpr int N = LfVec<T>::N, TPR = LF_HD / N, GPB = 256 / TPR, E = LF_BW_GCOL_E;
+  __shared__ float s_red[8][2 * LF_HD];
+  __shared__ __align__(16) float s_kv[E][2][LF_HD];  // the group's keys and values
+  __shared__ int s_g[E];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = threadIdx.x / TPR, pi = threadIdx.x % TPR;
+  const int neg = (P.G + E - 1) / E;
+  const long long units = (long long)P.B * P.H * neg * nch;
+  for (long long un = blockIdx.x; un < units; un += gridDim.x) {
+    const int c = (int)(un % nch);
+    const long long be = un / nch;
+    const int e0 = (int)(be % neg) * E;
+    const long long bh = be / neg;
+    const int h = (int)(bh % P.H), b = (int)(bh / P.H), d = P.dil[h], n = P.n;
+    const int ng = P.binfo[(size_t)b * LF_BI_WORDS + LF_BI_NG];
+    if (e0 >= ng) continue;  // (block-uniform; the reduce reads no partial past ng)
+    const int nb = min(E, ng - e0);
+    const int32_t *gl = P.gidx + (size_t)b * P.G + e0;
+    const size_t base = (size_t)bh * n * LF_HD;
+    for (int x = threadIdx.x; x < E * (LF_HD / 2); x += 256) {
+      const int e = x / (LF_HD / 2), cc = 2 * (x % (LF_HD / 2));
+      float2 kv = make_float2(0.f, 0.f), vv = make_float2(0.f, 0.f);
+      if (e < nb) {
+        const size_t src = base + (size_t)gl[e] * LF_HD + cc;
+        kv = LfIo<T>::ld2(ks + src);
+        vv = LfIo<T>::ld2(vs + src);
+      }
+      s_kv[e][0][cc] = kv.x;
+      s_kv[e][0][cc + 1] = kv.y;
+      s_kv[e][1][cc] = vv.x;
+      s_kv[e][1][cc + 1] = vv.y;
+    }
+    if (threadIdx.x < E) s_g[threadIdx.x] = (int)threadIdx.x < nb ? gl[threadIdx.x] : -1;
+    __syncthreads();
+    int gg[E];
+#pragma unroll
+    for (int e = 0; e < E; e++) gg[e] = s_g[e];
+    float ak[E][N], av[E][N];
+#pragma unroll
+    for (int e = 0; e < E; e++)
+#pragma unroll
+      for (int k = 0; k < N; k++) ak[e][k] = av[e][k] = 0.f;
+    const int32_t *m = P.mask + (size_t)b * n;
+    const int i0 = c * LF_BW_GCOL_ROWS, i1 = min(n, i0 + LF_BW_GCOL_ROWS);
+    for (int rr = 0; rr < LF_BW_GCOL_ROWS; rr += GPB) {
+      // the row's loads all issued together (none waits on a mask test)
+      const int i = i0 + rr + grp;
+      const int ic = i < i1 ? i : i1 - 1;
+      float q[N], go[N];
+      LfVec<T>::ld(qs + base + (size_t)ic * LF_HD + pi * N, q);
+      LfVec<T>::ld(dO + base + (size_t)ic * LF_HD + pi * N, go);
+      const size_t ir = (size_t)bh * n + ic;
+      const int mi = m[ic];
+      const float lse_i = lse[ir], dl_i = delta[ir];
+      const bool row_ok = i < i1 && mi == 1;
+#pragma unroll
+      for (int e = 0; e < E; e++) {
+        float sc = 0.f, dp = 0.f;
+#pragma unroll
+        for (int k = 0; k < N; k++) {
+          sc += q[k] * s_kv[e][0][pi * N + k];
+          dp += go[k] * s_kv[e][1][pi * N + k];
+        }
+        sc = lf_group_sum<TPR>(sc);
+        dp = lf_group_sum<TPR>(dp);
+        if (!row_ok || gg[e] < 0 || lf_in_window(i, gg[e], P.r, d, P.causal)) continue;
+        const float pr = exp2f(sc * P.scale_log2 - lse_i * LF_LOG2E);
+        const float ds = pr * (dp - dl_i) * P.scale;
+#pragma unroll
+        for (int k = 0; k < N; k++) {
+          ak[e][k] += ds * q[k];
+          av[e][k] += pr * go[k];
+        }
+      }
+    }
+    // per key: the groups of a warp, then the warps in order
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+      if (e >= nb) break;  // (block-uniform)
+#pragma unroll
+      for (int o = TPR; o < 32; o <<= 1)
+#pragma unroll
+        for (int k = 0; k < N; k++) {
+          ak[e][k] += __shfl_xor_sync(0xffffffffu, ak[e][k], o);
+          av[e][k] += __shfl_xor_sync(0xffffffffu, av[e][k], o);
+        }
+      if (lane < TPR)
+#pragma unroll
+        for (int k = 0; k < N; k++) {
+          s_red[warp][pi * N + k] = ak[e][k];
+          s_red[warp][LF_HD + pi * N + k] = av[e][k];
+        }
+      __syncthreads();
+      if (warp == 0) {
+        float *dst = part + (((size_t)bh * P.G + (e0 + e)) * nch + c) * 2 * LF_HD;
+        for (int x = lane; x < 2 * LF_HD; x += 32) {
+          float t = 0.f;
+          for (int w = 0; w < 8; w++) t += s_red[w][x];
+          dst[x] = t;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
 // dK_s[g] += sum of chunks; dV_s[g] likewise.  One block of LF_BW_RED_WARPS
 // warps per (b, h, e): warp w sums chunks w, w + LF_BW_RED_WARPS, ... in
 // order (four loads in flight), then the warps' sums are added in warp
@@ -816,10 +931,18 @@ static cudaError_t lf_bwd_global_parts(const LfLaunch &L, const LfTcBwdArgs &a, 
   e = cudaMemsetAsync(a.dqg, 0, (size_t)D.B * D.H * D.n * LF_HD * sizeof(T), L.stream);
   if (e != cudaSuccess) return e;
   if (D.G > 0) {
-    const long long wk = (long long)D.B * D.H * D.G * nchc, wr = (long long)D.B * D.H * D.G;
-    const unsigned ugrid = (unsigned)std::min<long long>(wk, 148LL * 16);  // grid-strided units
-    lf_bwd_gcol_kernel<T><<<ugrid, 256, 0, L.stream>>>(
-        D, (const T *)a.qs, (const T *)a.ks, (const T *)a.vs, a.lse, (const T *)a.dO, delta, part_kv, nchc);
+    const long long wr = (long long)D.B * D.H * D.G;
+    if (D.G >= LF_BW_GCOL_E) {  // several global keys: each row read once per group of keys
+      const long long wk = (long long)D.B * D.H * ((D.G + LF_BW_GCOL_E - 1) / LF_BW_GCOL_E) * nchc;
+      const unsigned ugrid = (unsigned)std::min<long long>(wk, 148LL * 16);  // grid-strided units
+      lf_bwd_gcol4_kernel<T><<<ugrid, 256, 0, L.stream>>>(
+          D, (const T *)a.qs, (const T *)a.ks, (const T *)a.vs, a.lse, (const T *)a.dO, delta, part_kv, nchc);
+    } else {
+      const long long wk = (long long)D.B * D.H * D.G * nchc;
+      const unsigned ugrid = (unsigned)std::min<long long>(wk, 148LL * 16);  // grid-strided units
+      lf_bwd_gcol_kernel<T><<<ugrid, 256, 0, L.stream>>>(
+          D, (const T *)a.qs, (const T *)a.ks, (const T *)a.vs, a.lse, (const T *)a.dO, delta, part_kv, nchc);
+    }
     const unsigned rgrid = (unsigned)std::min<long long>(wr, 4096);
     lf_bwd_gcol_reduce<T><<<rgrid, 32 * LF_BW_RED_WARPS, 0, L.stream>>>(D, part_kv, nchc, (T *)a.dks,
                                                                         (T *)a.dvs);

@@ -192,8 +192,9 @@ int lf_attn_status(void *workspace, void *stream);
  * Pass NULL, NULL to turn it off. */
 int lf_attn_set_timing_events(void *ev_start, void *ev_stop);
 
-/* Test hook for the device-side failure detection (SURVEY: failure
- * detection without a GPU fault).  Applies to the following lf_attn_fwd /
+/* Test hook for the device-side failure detection, exercised without any
+ * GPU fault: an expired bounded wait is made to happen on purpose.  Applies
+ * to the following lf_attn_fwd /
  * lf_attn_bwd calls of the calling thread until it is called again:
  *   wait_limit_us  the limit of every bounded device wait, in microseconds
  *                  (0 = the default 1.5 s);

@@ -100,7 +100,7 @@ __device__ __forceinline__ bool lf_wait_fast(uint32_t bar, uint32_t parity,
 }
 
 // Warp-uniform bounded wait: the converged warp polls together (every lane
-// acquires the phase itself), and the verdict is made uniform before the
+// acquires the phase itself), and the outcome is made uniform before the
 // warp-collective tcgen05 instructions that follow.
 __device__ __forceinline__ bool lf_wait_warp(uint32_t bar, uint32_t parity,
                                              volatile int *abort_flag, int32_t *status, int site) {

@@ -146,7 +146,7 @@ def job_throughput(units_per_rank: int, world: int, ms_per_step: float) -> float
 # DRAM traffic of the main forward kernel per launch, from the ncu captures
 # summarised under profiles/; reported only while the kernel sources are the
 # ones that were profiled (their sha256 prefix), else null.
-PROFILED_TRAFFIC = {"base_bf16": {"bytes": 31919872, "sha": "3a8a590cb9f161b1"}}
+PROFILED_TRAFFIC = {"base_bf16": {"bytes": 31919872, "sha": "e3273b3afd2a8e39"}}
 
 
 def kernel_traffic(workload: str):
